@@ -1,0 +1,78 @@
+// Shared device helpers for the GPT-2 training-step kernels (sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+typedef __nv_bfloat16 bf16;
+
+// Library-wide device error word.  Kernels never trap: a bounded wait that
+// gives up, or an out-of-range index, records a code here and the kernel
+// returns.  The host reads and clears it at its sync points.
+enum DeviceErr : int {
+  DERR_NONE = 0,
+  DERR_TOKEN_RANGE = 1,     // a token or target id >= padded vocab
+  DERR_WAIT_TIMEOUT = 2,    // an mbarrier wait ran past its limit
+  DERR_NONFINITE = 3,       // non-finite gradient norm (update skipped)
+};
+
+// (the library is one translation unit, so this is its single definition)
+__device__ int g_device_err = 0;
+
+__device__ __forceinline__ void set_device_err(int code) { atomicCAS(&g_device_err, 0, code); }
+
+// --------------------------------------------------------------- numerics
+__device__ __forceinline__ float bf2f(bf16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ bf16 f2bf(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(v);
+}
+
+// hardware tanh approximation (max rel. error ~2^-11), used where the result
+// is rounded to bf16 anyway
+__device__ __forceinline__ float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GELU, tanh form: 0.5*u*(1+tanh(sqrt(2/pi)*(u+0.044715*u^3)))
+#define GELU_K 0.7978845608028654f
+#define GELU_A 0.044715f
+template <bool FAST>
+__device__ __forceinline__ float gelu_tanh(float u) {
+  float t = GELU_K * (u + GELU_A * u * u * u);
+  float th = FAST ? tanh_fast(t) : tanhf(t);
+  return 0.5f * u * (1.0f + th);
+}
+template <bool FAST>
+__device__ __forceinline__ float gelu_tanh_grad(float u) {
+  float t = GELU_K * (u + GELU_A * u * u * u);
+  float th = FAST ? tanh_fast(t) : tanhf(t);
+  return 0.5f * (1.0f + th) + 0.5f * u * (1.0f - th * th) * GELU_K * (1.0f + 3.0f * GELU_A * u * u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+static inline int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }

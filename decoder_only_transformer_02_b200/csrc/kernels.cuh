@@ -1,0 +1,612 @@
+// Memory-bound kernels of the GPT-2 step: embedding, LayerNorm, softmax
+// cross-entropy, bias-gradient column sums, gradient norm, AdamW, init.
+// Every reduction runs in a fixed order (no floating-point atomics), so results
+// are bit-reproducible run to run.
+#pragma once
+#include "common.cuh"
+
+namespace k {
+
+template <typename T>
+__device__ __forceinline__ float ld_f(const T* p);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ld_f<bf16>(const bf16* p) { return bf2f(*p); }
+template <typename T>
+__device__ __forceinline__ void st_f(T* p, float v);
+template <>
+__device__ __forceinline__ void st_f<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void st_f<bf16>(bf16* p, float v) { *p = f2bf(v); }
+
+// ------------------------------------------------------------ embedding
+// x0[b,t,:] = wte[tok[b,t],:] + wpe[t,:]; an id >= V marks the error word and
+// the row is written as wpe only.  Also checks targets (may be null).
+__global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const int32_t* __restrict__ tgt,
+                                 const float* __restrict__ wte, const float* __restrict__ wpe, float* __restrict__ x,
+                                 int M, int T, int C, int V, int* __restrict__ bad) {
+  const int c4 = C / 4;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < (long)M * c4; i += (long)gridDim.x * blockDim.x) {
+    const int row = (int)(i / c4), c = (int)(i % c4);
+    const int id = tok[row];
+    const int t = row % T;
+    float4 p = reinterpret_cast<const float4*>(wpe + (long)t * C)[c];
+    if (id >= 0 && id < V) {
+      float4 w = reinterpret_cast<const float4*>(wte + (long)id * C)[c];
+      p.x += w.x;
+      p.y += w.y;
+      p.z += w.z;
+      p.w += w.w;
+    } else if (c == 0) {
+      atomicExch(bad, 1);
+    }
+    if (c == 0 && tgt != nullptr) {
+      const int y = tgt[row];
+      if (y < 0 || y >= V) atomicExch(bad, 1);
+    }
+    reinterpret_cast<float4*>(x + (long)row * C)[c] = p;
+  }
+}
+
+// single-CTA bitonic sort of the keys (token << 16 | position), n <= capacity
+// (a power of two, padded with 0xffffffff).  Sorting (token, position) pairs
+// gives every token's positions in ascending order: the fixed summation order
+// of the embedding scatter-add.
+// An id outside [0, V) sorts under the sentinel token 0xffff (never a valid
+// row: V <= 65472) and is skipped by the scatter.
+__global__ void sort_keys_kernel(const int32_t* __restrict__ tok, int M, int V, uint32_t* __restrict__ keys_out,
+                                 int cap) {
+  extern __shared__ uint32_t sk[];
+  for (int i = threadIdx.x; i < cap; i += blockDim.x) {
+    uint32_t key = 0xffffffffu;
+    if (i < M) {
+      const int t = tok[i];
+      key = ((t >= 0 && t < V) ? (uint32_t)t : 0xffffu) << 16 | (uint32_t)i;
+    }
+    sk[i] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= cap; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < cap / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = ((lo & size) == 0);
+        const uint32_t a = sk[lo], b = sk[hi];
+        if ((a > b) == up) {
+          sk[lo] = b;
+          sk[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < M; i += blockDim.x) keys_out[i] = sk[i];
+}
+
+// Stage 1 of the deterministic scatter-add.  Sorted entries are cut into
+// chunks of CH; chunk c sums each run of equal tokens it holds (positions in
+// ascending order) and writes the run's sum to part[first sorted index of the
+// run].  dx0 is fp32 [M, C]; one CTA per chunk, threads over columns.
+constexpr int EMB_CH = 32;
+__global__ void embed_bwd_partial_kernel(const uint32_t* __restrict__ keys, const float* __restrict__ dx, int M, int C,
+                                         float* __restrict__ part) {
+  const int c0 = blockIdx.x * EMB_CH;
+  const int c1 = min(M, c0 + EMB_CH);
+  for (int col = threadIdx.x; col < C; col += blockDim.x) {
+    int run_start = c0;
+    float acc = 0.f;
+    for (int s = c0; s < c1; ++s) {
+      const uint32_t key = keys[s];
+      acc += dx[(long)(key & 0xffffu) * C + col];
+      const bool last = (s + 1 == c1) || ((keys[s + 1] >> 16) != (key >> 16));
+      if (last) {
+        part[(long)run_start * C + col] = acc;
+        acc = 0.f;
+        run_start = s + 1;
+      }
+    }
+  }
+}
+
+// Stage 2: one CTA per sorted index that starts a token's segment; sums the
+// run partials of that segment (in sorted order) into dwte[token].
+__global__ void embed_bwd_reduce_kernel(const uint32_t* __restrict__ keys, const float* __restrict__ part, int M, int C,
+                                        int V, float* __restrict__ dwte) {
+  for (int s = blockIdx.x; s < M; s += gridDim.x) {
+    const uint32_t tokn = keys[s] >> 16;
+    if (tokn >= (uint32_t)V) continue;                   // out-of-range id (already flagged)
+    if (s > 0 && (keys[s - 1] >> 16) == tokn) continue;  // not a segment start
+    int e = s + 1;
+    while (e < M && (keys[e] >> 16) == tokn) ++e;
+    for (int col = threadIdx.x; col < C; col += blockDim.x) {
+      float acc = 0.f;
+      // run partials start at s and at each chunk boundary inside [s, e)
+      acc += part[(long)s * C + col];
+      for (int cb = (s / EMB_CH + 1) * EMB_CH; cb < e; cb += EMB_CH) acc += part[(long)cb * C + col];
+      dwte[(long)tokn * C + col] += acc;
+    }
+  }
+}
+
+// dwpe[t] += sum_b dx0[b,t]
+__global__ void wpe_bwd_kernel(const float* __restrict__ dx, int B, int T, int C, float* __restrict__ dwpe) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < (long)T * C; i += (long)gridDim.x * blockDim.x) {
+    const long t = i / C, c = i % C;
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b) acc += dx[((long)b * T + t) * C + c];
+    dwpe[t * C + c] += acc;
+  }
+}
+
+// ------------------------------------------------------------ LayerNorm
+// One warp per row, the row held in registers (C = 128 * NV), two-pass
+// mean/variance, biased variance, eps 1e-5.  Writes y (bf16 or fp32) and the
+// row's mean and rstd.
+template <int NV, typename TO>
+__global__ void ln_fwd_kernel(const float* __restrict__ x, const float* __restrict__ gam, const float* __restrict__ bet,
+                              TO* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int M) {
+  constexpr int C = 128 * NV;
+  const int lane = threadIdx.x & 31;
+  const long row = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5;
+  if (row >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * C);
+  float4 v[NV];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    v[i] = xr[lane + 32 * i];
+    s += v[i].x + v[i].y + v[i].z + v[i].w;
+  }
+  const float mu = warp_sum(s) * (1.f / C);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const float a = v[i].x - mu, b = v[i].y - mu, c = v[i].z - mu, d = v[i].w - mu;
+    q += a * a + b * b + c * c + d * d;
+  }
+  const float var = warp_sum(q) * (1.f / C);
+  const float rs = rsqrtf(var + 1e-5f);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = 4 * (lane + 32 * i);
+    const float4 gg = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
+    const float4 bb = reinterpret_cast<const float4*>(bet)[lane + 32 * i];
+    const float o0 = (v[i].x - mu) * rs * gg.x + bb.x;
+    const float o1 = (v[i].y - mu) * rs * gg.y + bb.y;
+    const float o2 = (v[i].z - mu) * rs * gg.z + bb.z;
+    const float o3 = (v[i].w - mu) * rs * gg.w + bb.w;
+    if constexpr (sizeof(TO) == 2) {
+      uint2 w = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+      *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * C + c) = w;
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * C + c) = make_float4(o0, o1, o2, o3);
+    }
+  }
+  if (lane == 0) {
+    mean[row] = mu;
+    rstd[row] = rs;
+  }
+}
+
+// LayerNorm backward fused with the residual stream.  One warp per row:
+//   dxhat = dy*g ; dx = rstd*(dxhat - mean(dxhat) - xhat*mean(dxhat*xhat))
+//   dres = (accumulate ? dres : 0) + dx     (fp32, in place)   and a bf16 copy
+// Per-block partial column sums (fixed row ranges, fixed order) of
+//   dy*xhat (-> dgamma), dy (-> dbeta), dres_out (-> the bias gradient of the
+//   linear layer whose output is this residual point).
+template <int NV, typename TI>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const TI* __restrict__ dy, const float* __restrict__ x,
+                                                     const float* __restrict__ mean, const float* __restrict__ rstd,
+                                                     const float* __restrict__ gam, float* __restrict__ dres,
+                                                     bf16* __restrict__ dres_bf, int M, int rows_per_block,
+                                                     int accumulate, float* __restrict__ part) {
+  constexpr int C = 128 * NV;
+  constexpr int WARPS = 8;
+  __shared__ float4 red[3 * C / 4];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float4 pg[NV], pb[NV], pd[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) pg[i] = pb[i] = pd[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 gv[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) gv[i] = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
+  const long r0 = (long)blockIdx.x * rows_per_block;
+  const long r1 = min((long)M, r0 + rows_per_block);
+  for (long row = r0 + warp; row < r1; row += WARPS) {
+    const float mu = mean[row], rs = rstd[row];
+    float4 xh[NV], dyv[NV];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * (lane + 32 * i);
+      const float4 xv = *reinterpret_cast<const float4*>(x + row * C + c);
+      xh[i] = make_float4((xv.x - mu) * rs, (xv.y - mu) * rs, (xv.z - mu) * rs, (xv.w - mu) * rs);
+      if constexpr (sizeof(TI) == 2) {
+        const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(dy) + row * C + c);
+        const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+        dyv[i] = make_float4(a.x, a.y, b.x, b.y);
+      } else {
+        dyv[i] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(dy) + row * C + c);
+      }
+      const float d0 = dyv[i].x * gv[i].x, d1 = dyv[i].y * gv[i].y, d2 = dyv[i].z * gv[i].z, d3 = dyv[i].w * gv[i].w;
+      s1 += d0 + d1 + d2 + d3;
+      s2 += d0 * xh[i].x + d1 * xh[i].y + d2 * xh[i].z + d3 * xh[i].w;
+    }
+    s1 = warp_sum(s1) * (1.f / C);
+    s2 = warp_sum(s2) * (1.f / C);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * (lane + 32 * i);
+      float4 o;
+      o.x = rs * (dyv[i].x * gv[i].x - s1 - xh[i].x * s2);
+      o.y = rs * (dyv[i].y * gv[i].y - s1 - xh[i].y * s2);
+      o.z = rs * (dyv[i].z * gv[i].z - s1 - xh[i].z * s2);
+      o.w = rs * (dyv[i].w * gv[i].w - s1 - xh[i].w * s2);
+      float4* dp = reinterpret_cast<float4*>(dres + row * C + c);
+      if (accumulate) {
+        const float4 r = *dp;
+        o.x += r.x;
+        o.y += r.y;
+        o.z += r.z;
+        o.w += r.w;
+      }
+      *dp = o;
+      if (dres_bf != nullptr)
+        *reinterpret_cast<uint2*>(dres_bf + row * C + c) = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+      pg[i].x += dyv[i].x * xh[i].x;
+      pg[i].y += dyv[i].y * xh[i].y;
+      pg[i].z += dyv[i].z * xh[i].z;
+      pg[i].w += dyv[i].w * xh[i].w;
+      pb[i].x += dyv[i].x;
+      pb[i].y += dyv[i].y;
+      pb[i].z += dyv[i].z;
+      pb[i].w += dyv[i].w;
+      pd[i].x += o.x;
+      pd[i].y += o.y;
+      pd[i].z += o.z;
+      pd[i].w += o.w;
+    }
+  }
+  // block reduction over warps, in warp order
+  for (int w = 0; w < WARPS; ++w) {
+    if (warp == w) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int c4 = lane + 32 * i;
+        float4 a = pg[i], b = pb[i], d = pd[i];
+        if (w > 0) {
+          const float4 ra = red[c4], rb = red[C / 4 + c4], rd = red[2 * (C / 4) + c4];
+          a = make_float4(ra.x + a.x, ra.y + a.y, ra.z + a.z, ra.w + a.w);
+          b = make_float4(rb.x + b.x, rb.y + b.y, rb.z + b.z, rb.w + b.w);
+          d = make_float4(rd.x + d.x, rd.y + d.y, rd.z + d.z, rd.w + d.w);
+        }
+        red[c4] = a;
+        red[C / 4 + c4] = b;
+        red[2 * (C / 4) + c4] = d;
+      }
+    }
+    __syncthreads();
+  }
+  const float* rf = reinterpret_cast<const float*>(red);
+  for (int idx = threadIdx.x; idx < 3 * C; idx += blockDim.x) part[(long)blockIdx.x * 3 * C + idx] = rf[idx];
+}
+
+// sum the per-block partials (fixed order) into dgamma, dbeta and, when given,
+// a bias gradient: out_k[c] += sum_blk part[blk][k][c]
+__global__ void ln_bwd_finish_kernel(const float* __restrict__ part, int nblk, int C, float* __restrict__ dg,
+                                     float* __restrict__ db, float* __restrict__ dbias) {
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < 3 * C; idx += gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int b = 0; b < nblk; ++b) acc += part[(long)b * 3 * C + idx];
+    const int which = idx / C, c = idx % C;
+    if (which == 0)
+      dg[c] += acc;
+    else if (which == 1)
+      db[c] += acc;
+    else if (dbias != nullptr)
+      dbias[c] += acc;
+  }
+}
+
+// column sums of an [M, N] matrix into out[N] (+=), two stages, fixed order
+template <typename T>
+__global__ void colsum_partial_kernel(const T* __restrict__ a, int M, int N, int rows_per_block,
+                                      float* __restrict__ part) {
+  const int r0 = blockIdx.y * rows_per_block;
+  const int r1 = min(M, r0 + rows_per_block);
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < N; c += gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int r = r0; r < r1; ++r) acc += ld_f(a + (long)r * N + c);
+    part[(long)blockIdx.y * N + c] = acc;
+  }
+}
+__global__ void colsum_finish_kernel(const float* __restrict__ part, int nblk, int N, float* __restrict__ out) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < N; c += gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int b = 0; b < nblk; ++b) acc += part[(long)b * N + c];
+    out[c] += acc;
+  }
+}
+
+// ------------------------------------------------------- cross-entropy
+// One CTA per row of logits z[M, V] (row kept in shared memory):
+//   lse = max + log(sum exp(z - max)); loss_row = lse - z[y]; argmax (lowest
+//   index among maxima).  When write_grad, the row is overwritten in place by
+//   dz = (exp(z - lse) - [j == y]) * gscale.
+template <typename T>
+__global__ void __launch_bounds__(1024) ce_kernel(T* __restrict__ z, const int32_t* __restrict__ y, int V,
+                                                  float* __restrict__ lse_out, float* __restrict__ loss_row,
+                                                  int32_t* __restrict__ amax_out, int write_grad, float gscale) {
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  T* row_s = reinterpret_cast<T*>(sm_raw);
+  __shared__ float red_v[32];
+  __shared__ int red_i[32];
+  __shared__ float red_s[32];
+  const long row = blockIdx.x;
+  T* zr = z + row * (long)V;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  // load the row (16-byte chunks) and find max / argmax
+  constexpr int EPC = 16 / sizeof(T);
+  const int nch = V / EPC;
+  float mx = -INFINITY;
+  int mi = 0x7fffffff;
+  for (int c = tid; c < nch; c += blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(zr)[c];
+    reinterpret_cast<uint4*>(row_s)[c] = u;
+    const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int i = 0; i < EPC; ++i) {
+      const float v = ld_f(e + i);
+      if (v > mx) {
+        mx = v;
+        mi = c * EPC + i;
+      }
+    }
+  }
+  for (int j = nch * EPC + tid; j < V; j += blockDim.x) {
+    const T v0 = zr[j];
+    row_s[j] = v0;
+    const float v = ld_f(&v0);
+    if (v > mx) {
+      mx = v;
+      mi = j;
+    }
+  }
+  // (max, lowest index) reduction
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, mx, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, mi, o);
+    if (ov > mx || (ov == mx && oi < mi)) {
+      mx = ov;
+      mi = oi;
+    }
+  }
+  if (lane == 0) {
+    red_v[warp] = mx;
+    red_i[warp] = mi;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    mx = lane < nw ? red_v[lane] : -INFINITY;
+    mi = lane < nw ? red_i[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, mx, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, mi, o);
+      if (ov > mx || (ov == mx && oi < mi)) {
+        mx = ov;
+        mi = oi;
+      }
+    }
+    if (lane == 0) {
+      red_v[0] = mx;
+      red_i[0] = mi;
+    }
+  }
+  __syncthreads();
+  mx = red_v[0];
+  const int amax = red_i[0];
+  // sum of exponentials
+  float se = 0.f;
+  for (int j = tid; j < V; j += blockDim.x) se += __expf(ld_f(row_s + j) - mx);
+  se = warp_sum(se);
+  if (lane == 0) red_s[warp] = se;
+  __syncthreads();
+  if (warp == 0) {
+    se = lane < nw ? red_s[lane] : 0.f;
+    se = warp_sum(se);
+    if (lane == 0) red_s[0] = se;
+  }
+  __syncthreads();
+  const float lse = mx + logf(red_s[0]);
+  const int tgt = y ? y[row] : -1;
+  if (tid == 0) {
+    if (lse_out) lse_out[row] = lse;
+    if (amax_out) amax_out[row] = amax;
+    if (loss_row) loss_row[row] = (tgt >= 0 && tgt < V) ? lse - ld_f(row_s + tgt) : 0.f;
+  }
+  if (write_grad) {
+    for (int j = tid; j < V; j += blockDim.x) {
+      float p = __expf(ld_f(row_s + j) - lse);
+      if (j == tgt) p -= 1.f;
+      st_f(zr + j, p * gscale);
+    }
+  }
+}
+
+// dz = (exp(z - lse) - onehot) * gscale in place, from the saved lse
+template <typename T>
+__global__ void ce_bwd_kernel(T* __restrict__ z, const int32_t* __restrict__ y, const float* __restrict__ lse, int V,
+                              float gscale) {
+  const long row = blockIdx.x;
+  T* zr = z + row * (long)V;
+  const float L = lse[row];
+  const int tgt = y[row];
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    float p = __expf(ld_f(zr + j) - L);
+    if (j == tgt) p -= 1.f;
+    st_f(zr + j, p * gscale);
+  }
+}
+
+// mean of the row losses into *loss (+= when accumulate), fixed order, 1 CTA
+__global__ void loss_mean_kernel(const float* __restrict__ rows, int M, float* __restrict__ loss, float* __restrict__ acc,
+                                 float acc_scale) {
+  __shared__ float red[32];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) s += rows[i];
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    s = warp_sum(s);
+    if (threadIdx.x == 0) {
+      const float m = s / (float)M;
+      *loss = m;
+      if (acc) *acc += m * acc_scale;
+    }
+  }
+}
+
+// ------------------------------------------------------------ optimizer
+// sum of squares of the flat gradient, stage 1: per-block partials (fixed
+// chunking: block b owns a contiguous range), fp64 accumulation
+__global__ void sumsq_partial_kernel(const float* __restrict__ g, long n, long per_block, double* __restrict__ part) {
+  __shared__ double red[32];
+  const long lo = blockIdx.x * per_block;
+  const long hi = min(n, lo + per_block);
+  double s = 0.0;
+  for (long i = lo + threadIdx.x * 4; i < hi; i += (long)blockDim.x * 4) {
+    if (i + 3 < hi) {
+      const float4 v = *reinterpret_cast<const float4*>(g + i);
+      s += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+    } else {
+      for (long j = i; j < hi; ++j) s += (double)g[j] * g[j];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    part[blockIdx.x] = t;
+  }
+}
+// stage 2, 1 CTA of 32 threads: out = [norm, clip scale, finite flag, bias
+// correction 1 - b1^t, bias correction 1 - b2^t]; the step counter t advances
+// only when the norm is finite (a non-finite norm skips the update).
+__global__ void norm_finish_kernel(const double* __restrict__ part, int nblk, float max_norm, float b1, float b2,
+                                   float* __restrict__ out, long long* __restrict__ step) {
+  double s = 0.0;
+  for (int i = threadIdx.x; i < nblk; i += 32) s += part[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (threadIdx.x == 0) {
+    const double n = sqrt(s);
+    const bool fin = isfinite(n);
+    out[0] = (float)n;
+    const double sc = (double)max_norm / (n + 1e-6);
+    out[1] = (float)(sc < 1.0 ? sc : 1.0);
+    out[2] = fin ? 1.f : 0.f;
+    long long t = *step;
+    if (fin) {
+      t += 1;
+      *step = t;
+    }
+    out[3] = (float)(1.0 - pow((double)b1, (double)t));
+    out[4] = (float)(1.0 - pow((double)b2, (double)t));
+  }
+}
+
+struct AdamSeg {
+  long begin;  // first flat index of a tensor (segments sorted, contiguous)
+  int decay;
+};
+
+// One launch over the whole flat arena.  Segment table in shared memory; each
+// thread handles 4 consecutive elements (every tensor size is a multiple of 4).
+//   g' = g * clip;  p *= (1 - lr*wd*decay);  m = b1 m + (1-b1) g';
+//   v = b2 v + (1-b2) g'^2;  p -= lr * (m / bc1) / (sqrt(v / bc2) + eps)
+// Skipped entirely (params untouched) when the norm is not finite.
+__global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
+                                                    float* __restrict__ m, float* __restrict__ v,
+                                                    bf16* __restrict__ pbf, long n, const AdamSeg* __restrict__ segs,
+                                                    int nseg, const float* __restrict__ normbuf, float lr, float wd,
+                                                    float b1, float b2, float eps) {
+  __shared__ long s_begin[160];
+  __shared__ int s_decay[160];
+  for (int i = threadIdx.x; i < nseg; i += blockDim.x) {
+    s_begin[i] = segs[i].begin;
+    s_decay[i] = segs[i].decay;
+  }
+  __syncthreads();
+  if (normbuf[2] == 0.f) return;
+  const float clip = normbuf[1];
+  const float bc1 = normbuf[3], bc2 = normbuf[4];
+  const float rbc2 = rsqrtf(bc2);
+  const float step = lr / bc1;
+  for (long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4; i < n; i += (long)gridDim.x * blockDim.x * 4) {
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_begin[mid] <= i)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    const float dec = s_decay[lo] ? (1.f - lr * wd) : 1.f;
+    float4 pv = *reinterpret_cast<float4*>(p + i);
+    const float4 gv = *reinterpret_cast<const float4*>(g + i);
+    float4 mv = *reinterpret_cast<float4*>(m + i);
+    float4 vv = *reinterpret_cast<float4*>(v + i);
+    float pa[4] = {pv.x, pv.y, pv.z, pv.w}, ga[4] = {gv.x, gv.y, gv.z, gv.w};
+    float ma[4] = {mv.x, mv.y, mv.z, mv.w}, va[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float gg = ga[e] * clip;
+      ma[e] = b1 * ma[e] + (1.f - b1) * gg;
+      va[e] = b2 * va[e] + (1.f - b2) * gg * gg;
+      const float denom = sqrtf(va[e]) * rbc2 + eps;
+      pa[e] = pa[e] * dec - step * ma[e] / denom;
+    }
+    *reinterpret_cast<float4*>(p + i) = make_float4(pa[0], pa[1], pa[2], pa[3]);
+    *reinterpret_cast<float4*>(m + i) = make_float4(ma[0], ma[1], ma[2], ma[3]);
+    *reinterpret_cast<float4*>(v + i) = make_float4(va[0], va[1], va[2], va[3]);
+    if (pbf != nullptr)
+      *reinterpret_cast<uint2*>(pbf + i) = make_uint2(pack_bf16x2(pa[0], pa[1]), pack_bf16x2(pa[2], pa[3]));
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ a, bf16* __restrict__ b, long n) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+    b[i] = f2bf(a[i]);
+}
+
+// ------------------------------------------------------------ init
+// counter-based N(0, std): splitmix64 of (seed, index) -> two uniforms ->
+// Box-Muller (cosine branch)
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  x += 0x9E3779B97F4A7C15ull;
+  x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+  x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+  return x ^ (x >> 31);
+}
+__global__ void init_normal_kernel(float* __restrict__ p, long n, uint64_t seed, long offset, float std) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const uint64_t h = splitmix64(seed * 0x2545F4914F6CDD1Dull + (uint64_t)(offset + i));
+    const float u1 = ((float)(h >> 40) + 1.f) * (1.f / 16777217.f);  // (0, 1]
+    const float u2 = (float)((h >> 16) & 0xFFFFFFu) * (1.f / 16777216.f);
+    p[i] = std * sqrtf(-2.f * logf(u1)) * cospif(2.f * u2);
+  }
+}
+__global__ void fill_kernel(float* __restrict__ p, long n, float v) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) p[i] = v;
+}
+
+}  // namespace k

@@ -1,0 +1,197 @@
+// Host-side runtime of the GPT-2 step: the handle, its device arenas and the
+// per-layer views into them.  Included by libgpt2.cu (single translation unit).
+#pragma once
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/gpt2.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "kernels.cuh"
+#include "simt_gemm.cuh"
+#include "tc_gemm.h"
+
+struct TensorInfo {
+  std::string name;
+  size_t offset;
+  size_t numel;
+  int rows, cols;  // cols == 0 for 1-D tensors
+  int decay;
+};
+
+struct LayerOffsets {
+  size_t ln1g, ln1b, attnw, attnb, projw, projb, ln2g, ln2b, fcw, fcb, mpw, mpb;
+};
+
+struct gpt2 {
+  gpt2_config cfg{};
+  int L = 0, H = 0, C = 0, V = 0, Vp = 0, P = 0, maxB = 0, maxT = 0, prec = 0;
+  size_t es = 4;  // bytes per activation element (2 in bf16 mode)
+  cudaStream_t stream = nullptr;
+  std::string err = "ok";
+  int64_t launches = 0;
+
+  // parameters, flat
+  std::vector<TensorInfo> tensors;
+  std::vector<LayerOffsets> lo;
+  size_t wte = 0, wpe = 0, lnfg = 0, lnfb = 0;
+  size_t nparams = 0;
+  float *params = nullptr, *grads = nullptr, *m = nullptr, *v = nullptr;
+  bf16* pbf = nullptr;  // bf16 copy of the weights (bf16 mode)
+  int64_t adam_t = 0;
+
+  // activations (element type: bf16 in bf16 mode, fp32 otherwise, unless noted)
+  float* res = nullptr;  // fp32 residual stream, (2L+1) points x [M, C]
+  uint8_t *ln1 = nullptr, *ln2 = nullptr;
+  float *ln1_mean = nullptr, *ln1_rstd = nullptr, *ln2_mean = nullptr, *ln2_rstd = nullptr;
+  uint8_t *qkv = nullptr, *att = nullptr, *fcu = nullptr, *fca = nullptr, *lnf = nullptr, *logits = nullptr;
+  float *lse = nullptr, *lnf_mean = nullptr, *lnf_rstd = nullptr;
+  float *ce_lse = nullptr, *losses = nullptr, *d_loss = nullptr;
+  int32_t* argmax = nullptr;
+
+  // backward scratch
+  float *dres = nullptr, *dln = nullptr, *attn_D = nullptr, *ln_part = nullptr, *cs_part = nullptr;
+  bf16* dres_bf = nullptr;
+  uint8_t *dbig = nullptr, *dqkv = nullptr, *datt = nullptr;
+  float* splitk_ws = nullptr;
+  size_t splitk_bytes = 0;
+  uint32_t* emb_keys = nullptr;
+  float* emb_part = nullptr;
+  int sort_cap = 0;
+
+  // optimizer
+  float* normbuf = nullptr;  // [norm, clip scale, finite flag, 1-b1^t, 1-b2^t]
+  long long* d_step = nullptr;  // AdamW step counter t (device)
+  double* norm_part = nullptr;
+  int norm_blocks = 0;
+  k::AdamSeg* segs = nullptr;
+  int nseg = 0;
+
+  int* d_bad = nullptr;  // token-range flag
+  int32_t *tok_dev = nullptr, *tgt_dev = nullptr;
+
+  // state of the last forward
+  int B = 0, T = 0;
+  bool have_fwd = false, have_targets = false, logits_valid = false, have_bwd_keys = false;
+  const int32_t* last_tok = nullptr;
+  const int32_t* last_tgt = nullptr;
+
+  long M() const { return (long)B * T; }
+  long Mmax() const { return (long)maxB * maxT; }
+  float* P32(size_t off) { return params + off; }
+  float* G32(size_t off) { return grads + off; }
+  const bf16* PBF(size_t off) { return pbf + off; }
+};
+
+static int set_err(gpt2* h, int code, const std::string& msg) {
+  if (h) h->err = msg;
+  return code;
+}
+
+#define CU_CHECK(h, call)                                                                         \
+  do {                                                                                            \
+    cudaError_t e_ = (call);                                                                      \
+    if (e_ != cudaSuccess) {                                                                      \
+      cudaGetLastError(); /* clear a non-sticky error so the handle stays usable */              \
+      return set_err((h), GPT2_ECUDA, std::string(#call) + ": " + cudaGetErrorString(e_));       \
+    }                                                                                             \
+  } while (0)
+
+#define LAUNCH_CHECK(h)                                                                           \
+  do {                                                                                            \
+    (h)->launches++;                                                                              \
+    cudaError_t e_ = cudaGetLastError();                                                          \
+    if (e_ != cudaSuccess)                                                                        \
+      return set_err((h), GPT2_ECUDA,                                                             \
+                     std::string("launch at ") + __FILE__ + ":" + std::to_string(__LINE__) + ": " +  \
+                         cudaGetErrorString(e_));                                                 \
+  } while (0)
+
+static int grid_for(long n, int threads, int cap_per_sm = 8) {
+  long b = (n + threads - 1) / threads;
+  long cap = 148L * cap_per_sm;
+  if (b > cap) b = cap;
+  if (b < 1) b = 1;
+  return (int)b;
+}
+
+static void build_tensor_table(gpt2* h) {
+  h->tensors.clear();
+  h->lo.assign(h->L, LayerOffsets{});
+  size_t off = 0;
+  auto add = [&](const std::string& n, int rows, int cols, int decay) -> size_t {
+    TensorInfo t;
+    t.name = n;
+    t.offset = off;
+    t.rows = rows;
+    t.cols = cols;
+    t.numel = (size_t)rows * (cols ? cols : 1);
+    t.decay = decay;
+    h->tensors.push_back(t);
+    off += t.numel;
+    return t.offset;
+  };
+  const int C = h->C;
+  h->wte = add("wte", h->Vp, C, 1);
+  h->wpe = add("wpe", h->P, C, 1);
+  for (int l = 0; l < h->L; ++l) {
+    const std::string p = "h" + std::to_string(l) + ".";
+    LayerOffsets& o = h->lo[l];
+    o.ln1g = add(p + "ln1.g", C, 0, 0);
+    o.ln1b = add(p + "ln1.b", C, 0, 0);
+    o.attnw = add(p + "attn.w", 3 * C, C, 1);
+    o.attnb = add(p + "attn.b", 3 * C, 0, 0);
+    o.projw = add(p + "proj.w", C, C, 1);
+    o.projb = add(p + "proj.b", C, 0, 0);
+    o.ln2g = add(p + "ln2.g", C, 0, 0);
+    o.ln2b = add(p + "ln2.b", C, 0, 0);
+    o.fcw = add(p + "fc.w", 4 * C, C, 1);
+    o.fcb = add(p + "fc.b", 4 * C, 0, 0);
+    o.mpw = add(p + "mproj.w", C, 4 * C, 1);
+    o.mpb = add(p + "mproj.b", C, 0, 0);
+  }
+  h->lnfg = add("lnf.g", C, 0, 0);
+  h->lnfb = add("lnf.b", C, 0, 0);
+  h->nparams = off;
+}
+
+static int dev_alloc(gpt2* h, void** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    return set_err(h, GPT2_ENOMEM, std::string("cudaMalloc(") + std::to_string(bytes) + "): " + cudaGetErrorString(e));
+  }
+  return GPT2_OK;
+}
+#define ALLOC(h, ptr, bytes)                                                    \
+  do {                                                                          \
+    int r_ = dev_alloc((h), reinterpret_cast<void**>(&(ptr)), (size_t)(bytes)); \
+    if (r_ != GPT2_OK) return r_;                                               \
+  } while (0)
+
+static void free_all(gpt2* h) {
+  void* ptrs[] = {h->params,  h->grads,   h->m,        h->v,        h->pbf,      h->res,      h->ln1,
+                  h->ln2,     h->ln1_mean, h->ln1_rstd, h->ln2_mean, h->ln2_rstd, h->qkv,      h->att,
+                  h->fcu,     h->fca,     h->lnf,      h->logits,   h->lse,      h->lnf_mean, h->lnf_rstd,
+                  h->ce_lse,  h->losses,  h->d_loss,   h->argmax,   h->dres,     h->dln,      h->attn_D,
+                  h->ln_part, h->cs_part, h->dres_bf,  h->dbig,     h->dqkv,     h->datt,     h->splitk_ws,
+                  h->emb_keys, h->emb_part, h->normbuf, h->d_step, h->norm_part, h->segs,    h->d_bad,    h->tok_dev,
+                  h->tgt_dev};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+// rows handled per CTA by the LayerNorm backward (multiple of 8 warps)
+static int ln_rows_per_block(long M) {
+  long r = (M + 295) / 296;
+  r = (r + 7) / 8 * 8;
+  return (int)(r < 8 ? 8 : r);
+}
+static int colsum_rows_per_block(long M) {
+  long r = (M + 127) / 128;
+  return (int)(r < 16 ? 16 : r);
+}

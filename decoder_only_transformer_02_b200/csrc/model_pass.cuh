@@ -1,0 +1,178 @@
+// The training step itself: forward, backward, clip + AdamW.
+#pragma once
+#include "model_create.cuh"
+
+struct Views {
+  gpt2* h;
+  float* res(int i) const { return h->res + (size_t)i * h->Mmax() * h->C; }
+  uint8_t* ln1(int l) const { return h->ln1 + (size_t)l * h->Mmax() * h->C * h->es; }
+  uint8_t* ln2(int l) const { return h->ln2 + (size_t)l * h->Mmax() * h->C * h->es; }
+  float* ln1m(int l) const { return h->ln1_mean + (size_t)l * h->Mmax(); }
+  float* ln1r(int l) const { return h->ln1_rstd + (size_t)l * h->Mmax(); }
+  float* ln2m(int l) const { return h->ln2_mean + (size_t)l * h->Mmax(); }
+  float* ln2r(int l) const { return h->ln2_rstd + (size_t)l * h->Mmax(); }
+  uint8_t* qkv(int l) const { return h->qkv + (size_t)l * h->Mmax() * 3 * h->C * h->es; }
+  uint8_t* att(int l) const { return h->att + (size_t)l * h->Mmax() * h->C * h->es; }
+  uint8_t* fcu(int l) const { return h->fcu + (size_t)l * h->Mmax() * 4 * h->C * h->es; }
+  uint8_t* fca(int l) const { return h->fca + (size_t)l * h->Mmax() * 4 * h->C * h->es; }
+};
+
+#define RET_IF(x)                \
+  do {                           \
+    int r__ = (x);               \
+    if (r__ != GPT2_OK) return r__; \
+  } while (0)
+
+// fuse: the softmax gradient (scaled by loss_scale / M) overwrites the logits
+// in the same pass that computes the loss
+static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, int T, bool fuse, float loss_scale) {
+  if (tok == nullptr) return set_err(h, GPT2_EINVAL, "tokens pointer is NULL");
+  if (B < 1 || T < 1 || B > h->maxB || T > h->maxT)
+    return set_err(h, GPT2_EINVAL, "B, T must satisfy 1 <= B <= max_B and 1 <= T <= max_T");
+  if (fuse && tgt == nullptr) return set_err(h, GPT2_EINVAL, "fused forward-backward needs targets");
+  h->B = B;
+  h->T = T;
+  h->have_fwd = false;
+  const long M = h->M();
+  const int C = h->C, L = h->L;
+  Views w{h};
+  // keep private copies of the ids: the backward pass reads them again
+  if (tok != h->tok_dev) CU_CHECK(h, cudaMemcpyAsync(h->tok_dev, tok, M * 4, cudaMemcpyDeviceToDevice, h->stream));
+  if (tgt && tgt != h->tgt_dev)
+    CU_CHECK(h, cudaMemcpyAsync(h->tgt_dev, tgt, M * 4, cudaMemcpyDeviceToDevice, h->stream));
+  const int32_t* dtgt = tgt ? h->tgt_dev : nullptr;
+
+  k::embed_fwd_kernel<<<grid_for(M * C / 4, 256), 256, 0, h->stream>>>(h->tok_dev, dtgt, h->P32(h->wte), h->P32(h->wpe),
+                                                                      w.res(0), (int)M, T, C, h->Vp, h->d_bad);
+  LAUNCH_CHECK(h);
+  for (int l = 0; l < L; ++l) {
+    const LayerOffsets& o = h->lo[l];
+    RET_IF(op_ln_fwd(h, w.res(2 * l), o.ln1g, o.ln1b, w.ln1(l), w.ln1m(l), w.ln1r(l), M));
+    RET_IF(op_lin_fwd(h, w.ln1(l), M, C, o.attnw, 3 * C, o.attnb, LIN_PLAIN, w.qkv(l), nullptr, nullptr));
+    RET_IF(op_attn_fwd(h, l));
+    RET_IF(op_lin_fwd(h, w.att(l), M, C, o.projw, C, o.projb, LIN_RESID, w.res(2 * l + 1), nullptr, w.res(2 * l)));
+    RET_IF(op_ln_fwd(h, w.res(2 * l + 1), o.ln2g, o.ln2b, w.ln2(l), w.ln2m(l), w.ln2r(l), M));
+    RET_IF(op_lin_fwd(h, w.ln2(l), M, C, o.fcw, 4 * C, o.fcb, LIN_GELU, w.fcu(l), w.fca(l), nullptr));
+    RET_IF(op_lin_fwd(h, w.fca(l), M, 4 * C, o.mpw, C, o.mpb, LIN_RESID, w.res(2 * l + 2), nullptr,
+                      w.res(2 * l + 1)));
+  }
+  RET_IF(op_ln_fwd(h, w.res(2 * L), h->lnfg, h->lnfb, h->lnf, h->lnf_mean, h->lnf_rstd, M));
+  // tied lm_head: logits = xf wte^T (no bias)
+  RET_IF(op_lin_fwd(h, h->lnf, M, C, h->wte, h->Vp, NO_OFF, LIN_NOBIAS, h->logits, nullptr, nullptr));
+  const size_t smem = (size_t)h->Vp * h->es;
+  const float gscale = loss_scale / (float)M;
+  if (h->prec == GPT2_BF16)
+    k::ce_kernel<bf16><<<(unsigned)M, 1024, smem, h->stream>>>((bf16*)h->logits, dtgt, h->Vp, h->ce_lse,
+                                                                dtgt ? h->losses : nullptr, h->argmax, fuse ? 1 : 0,
+                                                                gscale);
+  else
+    k::ce_kernel<float><<<(unsigned)M, 1024, smem, h->stream>>>((float*)h->logits, dtgt, h->Vp, h->ce_lse,
+                                                                 dtgt ? h->losses : nullptr, h->argmax, fuse ? 1 : 0,
+                                                                 gscale);
+  LAUNCH_CHECK(h);
+  if (dtgt) {
+    k::loss_mean_kernel<<<1, 1024, 0, h->stream>>>(h->losses, (int)M, h->d_loss, h->d_loss + 1,
+                                                   fuse ? loss_scale : 0.f);
+    LAUNCH_CHECK(h);
+  }
+  h->have_fwd = true;
+  h->have_targets = dtgt != nullptr;
+  h->logits_valid = !fuse;
+  return GPT2_OK;
+}
+
+static int backward_impl(gpt2* h, float loss_scale, bool fused) {
+  if (!h->have_fwd || !h->have_targets)
+    return set_err(h, GPT2_ESTATE, "backward needs a preceding forward with targets");
+  if (!fused && !h->logits_valid) return set_err(h, GPT2_ESTATE, "the logits of the last forward were consumed");
+  const long M = h->M();
+  const int C = h->C, L = h->L, B = h->B, T = h->T;
+  Views w{h};
+  if (!fused) {
+    const float gscale = loss_scale / (float)M;
+    if (h->prec == GPT2_BF16)
+      k::ce_bwd_kernel<bf16><<<(unsigned)M, 512, 0, h->stream>>>((bf16*)h->logits, h->tgt_dev, h->ce_lse, h->Vp,
+                                                                 gscale);
+    else
+      k::ce_bwd_kernel<float><<<(unsigned)M, 512, 0, h->stream>>>((float*)h->logits, h->tgt_dev, h->ce_lse, h->Vp,
+                                                                  gscale);
+    LAUNCH_CHECK(h);
+    h->logits_valid = false;
+  }
+  const void* dlog = h->logits;
+  const bool bf = h->prec == GPT2_BF16;
+  const void* dres_act = bf ? (const void*)h->dres_bf : (const void*)h->dres;
+  // lm_head (tied): dwte += dlogits^T xf ; dxf = dlogits wte
+  RET_IF(op_lin_wgrad(h, dlog, M, h->Vp, h->lnf, C, h->wte));
+  RET_IF(op_lin_dgrad(h, dlog, M, h->Vp, h->wte, C, DG_F32, h->dln, nullptr));
+  RET_IF(op_ln_bwd(h, h->dln, w.res(2 * L), h->lnf_mean, h->lnf_rstd, h->lnfg, h->lnfb, h->lo[L - 1].mpb, M, 0));
+  for (int l = L - 1; l >= 0; --l) {
+    const LayerOffsets& o = h->lo[l];
+    // MLP half: x_out = x_mid + mproj(gelu(fc(ln2(x_mid))))
+    RET_IF(op_lin_wgrad(h, dres_act, M, C, w.fca(l), 4 * C, o.mpw));
+    RET_IF(op_lin_dgrad(h, dres_act, M, C, o.mpw, 4 * C, DG_DGELU, h->dbig, w.fcu(l)));
+    RET_IF(op_colsum(h, h->dbig, M, 4 * C, o.fcb));
+    RET_IF(op_lin_wgrad(h, h->dbig, M, 4 * C, w.ln2(l), C, o.fcw));
+    RET_IF(op_lin_dgrad(h, h->dbig, M, 4 * C, o.fcw, C, DG_F32, h->dln, nullptr));
+    RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l + 1), w.ln2m(l), w.ln2r(l), o.ln2g, o.ln2b, o.projb, M, 1));
+    // attention half: x_mid = x_in + proj(attn(qkv(ln1(x_in))))
+    RET_IF(op_lin_wgrad(h, dres_act, M, C, w.att(l), C, o.projw));
+    RET_IF(op_lin_dgrad(h, dres_act, M, C, o.projw, C, DG_ACT, h->datt, nullptr));
+    RET_IF(op_attn_bwd(h, l));
+    RET_IF(op_colsum(h, h->dqkv, M, 3 * C, o.attnb));
+    RET_IF(op_lin_wgrad(h, h->dqkv, M, 3 * C, w.ln1(l), C, o.attnw));
+    RET_IF(op_lin_dgrad(h, h->dqkv, M, 3 * C, o.attnw, C, DG_F32, h->dln, nullptr));
+    RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l), w.ln1m(l), w.ln1r(l), o.ln1g, o.ln1b, l > 0 ? h->lo[l - 1].mpb : NO_OFF,
+                     M, 1));
+  }
+  // embeddings: dwte[tok] += dx0 (sorted, fixed order), dwpe[t] += sum_b dx0[b, t]
+  k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->stream>>>(h->tok_dev, (int)M, h->Vp, h->emb_keys,
+                                                                        h->sort_cap);
+  LAUNCH_CHECK(h);
+  const int eth = C < 256 ? C : 256;
+  k::embed_bwd_partial_kernel<<<(unsigned)((M + k::EMB_CH - 1) / k::EMB_CH), eth, 0, h->stream>>>(
+      h->emb_keys, h->dres, (int)M, C, h->emb_part);
+  LAUNCH_CHECK(h);
+  k::embed_bwd_reduce_kernel<<<grid_for(M, 1, 16), eth, 0, h->stream>>>(h->emb_keys, h->emb_part, (int)M, C,
+                                                                        h->Vp, h->G32(h->wte));
+  LAUNCH_CHECK(h);
+  k::wpe_bwd_kernel<<<grid_for((long)T * C, 256), 256, 0, h->stream>>>(h->dres, B, T, C, h->G32(h->wpe));
+  LAUNCH_CHECK(h);
+  h->have_bwd_keys = true;
+  h->have_targets = false;  // one backward per forward
+  return GPT2_OK;
+}
+
+static int adamw_impl(gpt2* h, float lr, float wd, float b1, float b2, float eps, float clip) {
+  const long n = (long)h->nparams;
+  long per = (n + h->norm_blocks - 1) / h->norm_blocks;
+  per = (per + 3) / 4 * 4;
+  k::sumsq_partial_kernel<<<h->norm_blocks, 256, 0, h->stream>>>(h->grads, n, per, h->norm_part);
+  LAUNCH_CHECK(h);
+  k::norm_finish_kernel<<<1, 32, 0, h->stream>>>(h->norm_part, h->norm_blocks, clip, b1, b2, h->normbuf, h->d_step);
+  LAUNCH_CHECK(h);
+  k::adamw_kernel<<<grid_for(n / 4, 256, 4), 256, 0, h->stream>>>(h->params, h->grads, h->m, h->v,
+                                                                  h->prec == GPT2_BF16 ? h->pbf : nullptr, n, h->segs,
+                                                                  h->nseg, h->normbuf, lr, wd, b1, b2, eps);
+  LAUNCH_CHECK(h);
+  return GPT2_OK;
+}
+
+// Sync point: surface device-side flags (token range, bounded-wait timeouts).
+static int check_device_flags(gpt2* h) {
+  CU_CHECK(h, cudaStreamSynchronize(h->stream));
+  int bad = 0;
+  CU_CHECK(h, cudaMemcpy(&bad, h->d_bad, 4, cudaMemcpyDeviceToHost));
+  int derr = 0;
+  CU_CHECK(h, cudaMemcpyFromSymbol(&derr, g_device_err, 4));
+  if (derr) {
+    int zero = 0;
+    cudaMemcpyToSymbol(g_device_err, &zero, 4);
+    return set_err(h, GPT2_ECUDA, "a device-side wait timed out (error code " + std::to_string(derr) + ")");
+  }
+  if (bad) {
+    CU_CHECK(h, cudaMemset(h->d_bad, 0, 4));
+    return set_err(h, GPT2_ETOKEN, "a token or target id lies outside [0, padded_vocab)");
+  }
+  return GPT2_OK;
+}

@@ -1,0 +1,601 @@
+// bf16 GEMM on the 5th-generation tensor cores (tcgen05) for sm_100a.
+//
+//   D[M,N] = sum_k A[m,k] * B[n,k]      (bf16 operands, fp32 accumulation)
+//
+// with the epilogue fused (bias, GELU, GELU', residual add, gradient
+// accumulation, split-K partials).  Every matrix product of the GPT-2 step is
+// one of three forms of this contraction:
+//   forward  Y = X W^T        A = X  [M,K] K-major   B = W  [N,K] K-major
+//   dgrad   dX = dY W         A = dY [M,N] K-major   B = W  viewed [K,N] MN-major
+//   wgrad   dW += dY^T X      A = dY viewed MN-major B = X  viewed MN-major
+// ("K-major": the contraction index is contiguous in memory; "MN-major": the
+// output index is contiguous.)  Both layouts are read straight from global
+// memory by TMA with the 128-byte swizzle; no transposed copy is ever made.
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: fills a ring of shared-memory stages (A tile
+//               128x64, B tile BNx64 per stage) and signals an mbarrier.
+//   warp 1      allocates TMEM and issues tcgen05.mma (one thread): 4 MMAs of
+//               128xBNx16 per stage; tcgen05.commit frees the stage and, at the
+//               end of a tile, marks the accumulator ready.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
+//               row), fused math, vectorised global stores.  Two accumulator
+//               buffers in TMEM let the epilogue of tile i overlap the MMAs of
+//               tile i+1.
+// Every mbarrier wait is bounded (about two seconds); a wait that gives up
+// records an error in g_device_err and the kernel drains its own in-flight
+// copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include "common.cuh"
+#include "tc_gemm.h"
+
+namespace tcg {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+template <int BN>
+struct Layout {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
+};
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 255u) == 255u && globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bit.
+//  K-major : rows of 128 B (64 bf16 along K); 8-row groups 1024 B apart (SBO).
+//  MN-major: rows of 128 B (64 bf16 along M or N), one row per K index;
+//            8-row K groups 1024 B apart (SBO); 64-wide M/N chunks 8 KB apart (LBO).
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, int mn_major) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((mn_major ? (8192u >> 4) : 1u) & 0x3FFFu) << 16;
+  d |= (uint64_t)((1024u >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor for kind::f16: bf16 x bf16 -> fp32, M=128, N=BN.
+template <int BN>
+__device__ __forceinline__ uint32_t make_idesc(int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void decode_tile(const Params& p, int tile, int& mb, int& nb, int& split) {
+  int per_split = p.num_m * p.num_n;
+  split = tile / per_split;
+  int t = tile - split * per_split;
+  mb = t % p.num_m;
+  nb = t / p.num_m;
+}
+
+// ------------------------------------------------------------- epilogue
+template <bool FULL>
+__device__ __forceinline__ void epi_store(const Params& p, int row, int col0, int split, const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  const long base = (long)row * p.ldc + col0;
+  if (p.bias != nullptr && p.epi != EPI_DGELU && p.epi != EPI_ACCUM_F32 && p.epi != EPI_PARTIAL_F32) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (FULL || col0 + i < p.N) v[i] += __ldg(p.bias + col0 + i);
+  }
+  switch (p.epi) {
+    case EPI_BF16: {
+      bf16* o = reinterpret_cast<bf16*>(p.out) + base;
+      if (FULL) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 w = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                               pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+          *reinterpret_cast<uint4*>(o + i) = w;
+        }
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.N) o[i] = f2bf(v[i]);
+      }
+    } break;
+    case EPI_F32: {
+      float* o = reinterpret_cast<float*>(p.out) + base;
+      if (FULL) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.N) o[i] = v[i];
+      }
+    } break;
+    case EPI_RESID_F32:
+    case EPI_ACCUM_F32: {
+      const float* rs = (p.epi == EPI_RESID_F32 ? p.resid : reinterpret_cast<const float*>(p.out)) + base;
+      float* o = reinterpret_cast<float*>(p.out) + base;
+      if (FULL) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float4 x = *reinterpret_cast<const float4*>(rs + i);
+          *reinterpret_cast<float4*>(o + i) = make_float4(x.x + v[i], x.y + v[i + 1], x.z + v[i + 2], x.w + v[i + 3]);
+        }
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.N) o[i] = rs[i] + v[i];
+      }
+    } break;
+    case EPI_GELU: {
+      bf16* o = reinterpret_cast<bf16*>(p.out) + base;
+      bf16* o2 = p.out2 + base;
+      if (FULL) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float u[8], g[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            u[j] = bf2f(f2bf(v[i + j]));  // the stored pre-activation, as rounded
+            g[j] = gelu_tanh<true>(u[j]);
+          }
+          *reinterpret_cast<uint4*>(o + i) = make_uint4(pack_bf16x2(u[0], u[1]), pack_bf16x2(u[2], u[3]),
+                                                        pack_bf16x2(u[4], u[5]), pack_bf16x2(u[6], u[7]));
+          *reinterpret_cast<uint4*>(o2 + i) = make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]),
+                                                         pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
+        }
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.N) {
+            float u = bf2f(f2bf(v[i]));
+            o[i] = f2bf(u);
+            o2[i] = f2bf(gelu_tanh<true>(u));
+          }
+      }
+    } break;
+    case EPI_DGELU: {
+      bf16* o = reinterpret_cast<bf16*>(p.out) + base;
+      const bf16* ua = p.aux + base;
+      if (FULL) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 uu = *reinterpret_cast<const uint4*>(ua + i);
+          uint32_t uw[4] = {uu.x, uu.y, uu.z, uu.w};
+          float d[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float2 f = unpack_bf16x2(uw[j]);
+            d[2 * j] = v[i + 2 * j] * gelu_tanh_grad<true>(f.x);
+            d[2 * j + 1] = v[i + 2 * j + 1] * gelu_tanh_grad<true>(f.y);
+          }
+          *reinterpret_cast<uint4*>(o + i) = make_uint4(pack_bf16x2(d[0], d[1]), pack_bf16x2(d[2], d[3]),
+                                                        pack_bf16x2(d[4], d[5]), pack_bf16x2(d[6], d[7]));
+        }
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.N) o[i] = f2bf(v[i] * gelu_tanh_grad<true>(bf2f(ua[i])));
+      }
+    } break;
+    case EPI_PARTIAL_F32: {
+      float* o = p.partial + (long)split * p.M * p.ldc + base;
+      if (FULL) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.N) o[i] = v[i];
+      }
+    } break;
+    default:
+      break;
+  }
+}
+
+// --------------------------------------------------------------- kernel
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                   const Params p) {
+  using L = Layout<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* empty = full + L::STAGES;
+  uint64_t* tfull = empty + L::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)L::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tma_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tma_b)) : "memory");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+        int mb, nb, split;
+        decode_tile(p, tile, mb, nb, split);
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % L::STAGES;
+          const uint32_t ph = (it / L::STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u)) {
+            set_device_err(DERR_WAIT_TIMEOUT);
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], L::STAGE_BYTES);
+          const uint32_t a_dst = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_dst = a_dst + L::A_BYTES;
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tma_load_2d(a_dst, &tma_a, k0, mb * BM, &full[s]);
+          } else {
+            tma_load_2d(a_dst, &tma_a, mb * BM, k0, &full[s]);
+            tma_load_2d(a_dst + 8192, &tma_a, mb * BM + 64, k0, &full[s]);
+          }
+          if (!p.b_mn) {
+            tma_load_2d(b_dst, &tma_b, k0, nb * BN, &full[s]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, &tma_b, nb * BN + 64 * j, k0, &full[s]);
+          }
+        }
+      }
+      // drain: every issued stage load has landed before the CTA exits
+      const uint32_t issued = it;
+      for (int s = 0; s < L::STAGES; ++s) {
+        if ((uint32_t)s < issued) {
+          const uint32_t last = issued - 1 - ((issued - 1 - s) % L::STAGES);
+          if (!mbar_wait(&full[s], (last / L::STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      const uint32_t idesc = make_idesc<BN>(p.a_mn, p.b_mn);
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tc) {
+        int mb, nb, split;
+        decode_tile(p, tile, mb, nb, split);
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+        const uint32_t buf = tc & 1u;
+        if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1u) ^ 1u)) {
+          set_device_err(DERR_WAIT_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % L::STAGES;
+          const uint32_t ph = (it / L::STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph)) {
+            set_device_err(DERR_WAIT_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + L::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = make_sdesc(a_addr + (p.a_mn ? k * 2048 : k * 32), p.a_mn);
+            const uint64_t bd = make_sdesc(b_addr + (p.b_mn ? k * 2048 : k * 32), p.b_mn);
+            tc_mma(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&tfull[buf]);
+      }
+      // drain: all MMAs issued by this thread have completed
+      tc_commit(drain);
+      if (!mbar_wait(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t tc = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tc) {
+      int mb, nb, split;
+      decode_tile(p, tile, mb, nb, split);
+      const uint32_t buf = tc & 1u;
+      if (!mbar_wait(&tfull[buf], (tc >> 1) & 1u)) {
+        set_device_err(DERR_WAIT_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int row = mb * BM + q * 32 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+#pragma unroll 1
+      for (int j = 0; j < BN / 32; ++j) {
+        uint32_t r[32];
+        tmem_ld32(tbase + j * 32, r);
+        tmem_wait_ld();
+        const int col0 = nb * BN + j * 32;
+        if (row < p.M && col0 < p.N) {
+          if (col0 + 32 <= p.N)
+            epi_store<true>(p, row, col0, split, r);
+          else
+            epi_store<false>(p, row, col0, split, r);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)L::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// Deterministic split-K reduction: out[i] += sum_s partial[s][i] (fixed order).
+__global__ void splitk_reduce_kernel(float* __restrict__ out, const float* __restrict__ partial, long n4, long stride,
+                                     int splits) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(out)[i];
+    for (int s = 0; s < splits; ++s) {
+      float4 v = reinterpret_cast<const float4*>(partial + s * stride)[i];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    reinterpret_cast<float4*>(out)[i] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ host
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
+// rows `ld` elements apart; box box_inner x box_outer; 128-byte swizzle.
+static int make_tmap(CUtensorMap* m, const void* base, long inner, long outer, long ld, int box_inner,
+                     int box_outer) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return -1;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int BN>
+static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid, cudaStream_t st) {
+  using L = Layout<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  tc_gemm_kernel<BN><<<grid, 192, L::SMEM_BYTES, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+int choose_splits(int tiles, int kb_total) {
+  const int sms = num_sms();
+  if (tiles >= sms) return 1;
+  int best = 1;
+  double best_eff = (double)tiles / (double)(((tiles + sms - 1) / sms) * sms);
+  for (int s = 2; s <= 16; ++s) {
+    if (kb_total / s < 4) break;
+    const int t = tiles * s;
+    const double eff = (double)t / (double)(((t + sms - 1) / sms) * sms);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+size_t splitk_workspace_bytes(int M, int N, int K, int bn) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (bn != 128) bn = (N <= 128) ? 128 : 256;
+  const int tiles = ceil_div(M, BM) * ceil_div(N, bn);
+  const int kbt = ceil_div(K, BK);
+  const int s = choose_splits(tiles, kbt);
+  return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
+}
+
+int gemm(const GemmArgs& g, cudaStream_t st) {
+  // shape / layout checks (TMA needs 16-byte row strides and base addresses)
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return -1;
+  if ((g.lda % 8) || (g.ldb % 8) || (g.ldc % 8)) return -1;
+  if ((reinterpret_cast<uintptr_t>(g.A) & 15) || (reinterpret_cast<uintptr_t>(g.B) & 15) ||
+      (reinterpret_cast<uintptr_t>(g.out) & 15))
+    return -1;
+  const int bn = (g.bn == 128 || g.N <= 128) ? 128 : 256;
+  CUtensorMap ta, tb;
+  if (!g.a_mn) {
+    if (make_tmap(&ta, g.A, g.K, g.M, g.lda, 64, BM)) return -2;
+  } else {
+    if (make_tmap(&ta, g.A, g.M, g.K, g.lda, 64, 64)) return -2;
+  }
+  if (!g.b_mn) {
+    if (make_tmap(&tb, g.B, g.K, g.N, g.ldb, 64, bn)) return -2;
+  } else {
+    if (make_tmap(&tb, g.B, g.N, g.K, g.ldb, 64, 64)) return -2;
+  }
+  Params p{};
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.a_mn = g.a_mn;
+  p.b_mn = g.b_mn;
+  p.num_m = ceil_div(g.M, BM);
+  p.num_n = ceil_div(g.N, bn);
+  p.kb_total = ceil_div(g.K, BK);
+  p.epi = g.epi;
+  p.bias = g.bias;
+  p.resid = g.resid;
+  p.out = g.out;
+  p.out2 = g.out2;
+  p.aux = g.aux;
+  p.ldc = g.ldc;
+  int splits = 1;
+  if (g.epi == EPI_ACCUM_F32 && g.workspace != nullptr) {
+    splits = choose_splits(p.num_m * p.num_n, p.kb_total);
+    if (splits > 1 && g.workspace_bytes < (size_t)splits * g.M * g.ldc * sizeof(float)) splits = 1;
+  }
+  if (splits > 1 && g.ldc != g.N) splits = 1;
+  if (splits > 1) {
+    const int kps = ceil_div(p.kb_total, splits);
+    splits = ceil_div(p.kb_total, kps);
+    p.kb_per_split = kps;
+    p.splits = splits;
+    p.epi = EPI_PARTIAL_F32;
+    p.partial = g.workspace;
+  } else {
+    p.kb_per_split = p.kb_total;
+    p.splits = 1;
+  }
+  p.total_tiles = p.num_m * p.num_n * p.splits;
+  const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
+  cudaError_t e = (bn == 128) ? launch<128>(ta, tb, p, grid, st) : launch<256>(ta, tb, p, grid, st);
+  if (e != cudaSuccess) return -3;
+  if (splits > 1) {
+    const long n = (long)g.M * g.N;
+    const long n4 = n / 4;
+    int blocks = (int)((n4 + 255) / 256);
+    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+    splitk_reduce_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(g.out), g.workspace, n4, n, splits);
+    if (cudaGetLastError() != cudaSuccess) return -3;
+  }
+  return 0;
+}
+
+}  // namespace tcg

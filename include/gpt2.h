@@ -1,0 +1,179 @@
+/* libgpt2: one GPT-2 training step on one NVIDIA B200 (sm_100a).
+ *
+ * C ABI: plain pointers and sizes only.  "d_" arguments are device pointers
+ * (CUDA global memory on the current device), "h_" arguments host pointers.
+ * Every call returns a status code (GPT2_OK = 0 or a negative GPT2_E*) unless
+ * documented otherwise; gpt2_last_error() gives a one-line reason.  Calls are
+ * asynchronous on the handle's stream unless an h_ output is requested, which
+ * synchronises that stream.
+ *
+ * The method (the pages it is described on):
+ *  - "Let's reproduce GPT-2 (124M)", video summary, Key Takeaways: the
+ *    architecture bullet (decoder-only, pre-LayerNorm, extra final LayerNorm,
+ *    GELU, 12 layers x 768 channels, vocab 50,257, seq 1024), the
+ *    hyperparameter bullet (AdamW betas 0.9/0.95, eps 1e-8, clip 1.0, weight
+ *    decay 0.1 on 2D tensors, warmup + cosine LR), the accumulation bullet
+ *    (loss divided by the number of micro-steps) and the weight tying /
+ *    padding bullet (tied wte/lm_head, vocab padded 50257 -> 50304).
+ *  - "Let's reproduce GPT-2 (124M)", video page, Chapters: cross entropy
+ *    loss; parameter sharing wte and lm_head; model initialization (std 0.02,
+ *    residual init); AdamW, gradient clipping; gradient accumulation.
+ *  - "From Scratch: Building GPT-2 for Efficient Language Modeling", Key
+ *    Features (token + positional embeddings, attention, GELU MLP, residuals)
+ *    and Training Setup table.
+ *
+ * Flat parameter order (also the order of grads, AdamW moments and
+ * checkpoints), every Linear weight stored [out, in] row-major:
+ *   wte[Vp, C], wpe[block, C];
+ *   per layer l: ln1.g[C], ln1.b[C], attn.w[3C, C], attn.b[3C], proj.w[C, C],
+ *                proj.b[C], ln2.g[C], ln2.b[C], fc.w[4C, C], fc.b[4C],
+ *                mproj.w[C, 4C], mproj.b[C];
+ *   lnf.g[C], lnf.b[C].
+ */
+#ifndef GPT2_B200_H
+#define GPT2_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPT2_OK 0
+#define GPT2_EINVAL (-1)     /* bad argument: null pointer, size out of range, unsupported shape */
+#define GPT2_ECUDA (-2)      /* a CUDA runtime call or kernel launch failed, or a device wait timed out */
+#define GPT2_ETOKEN (-3)     /* a token or target id outside [0, padded_vocab) (flagged on the device) */
+#define GPT2_ENOMEM (-4)     /* device or host allocation failed */
+#define GPT2_ESTATE (-5)     /* call out of order (e.g. backward without a forward with targets) */
+#define GPT2_ENONFINITE (-6) /* non-finite gradient norm: the AdamW update was skipped */
+
+#define GPT2_FP32 0 /* fp32 everywhere, CUDA-core (FFMA) matmuls: the parity mode */
+#define GPT2_BF16 1 /* bf16 tensor-core matmuls and attention, fp32 master weights,
+                       fp32 residual stream, fp32 LayerNorm statistics, LSE and loss */
+
+typedef struct {
+  int n_layer;      /* number of blocks L */
+  int n_head;       /* attention heads H (head dim C/H; must be 64 in BF16 mode) */
+  int n_embd;       /* channels C (multiple of 128, at most 1024) */
+  int vocab_size;   /* real vocabulary (targets must lie below it in practice) */
+  int padded_vocab; /* rows of wte = logits columns Vp (multiple of 64, at most 65472; 51200 in FP32 mode) */
+  int block_size;   /* maximum sequence length (rows of wpe) */
+  int max_B;        /* largest micro-batch the activations are sized for */
+  int max_T;        /* largest sequence length the activations are sized for (<= block_size) */
+  int precision;    /* GPT2_FP32 or GPT2_BF16 */
+} gpt2_config;
+
+typedef struct gpt2 gpt2_t; /* opaque; the library owns every device buffer it allocates */
+
+/* Allocate parameters, gradients, AdamW moments and activations on the
+ * current device and initialise the weights on the device from `seed`
+ * (counter-based normal generator): matrices and embeddings N(0, 0.02), the two
+ * residual projections N(0, 0.02/sqrt(2L)), biases 0, LayerNorm gains 1 and
+ * shifts 0 ("Let's reproduce GPT-2 (124M)", Chapters: model initialization).
+ * Gradients and moments start at zero.  *out receives the handle. */
+int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_t** out);
+/* Free everything the handle owns (synchronises its stream).  NULL is a no-op. */
+void gpt2_destroy(gpt2_t* h);
+/* Enqueue all later work on `cuda_stream` (a cudaStream_t; NULL = legacy default stream). */
+int gpt2_set_stream(gpt2_t* h, void* cuda_stream);
+
+/* Forward pass on d_tokens[B*T] (int32, row-major [B, T], device memory the
+ * caller keeps alive until the stream reaches it).  With d_targets non-NULL,
+ * also the mean softmax cross-entropy over all B*T positions and all Vp
+ * columns, the per-row argmax, and the state that gpt2_backward needs; with
+ * NULL, logits only.  B <= max_B, T <= max_T.  h_loss non-NULL: the loss is
+ * copied out (syncs; an out-of-range id then returns GPT2_ETOKEN). */
+int gpt2_forward(gpt2_t* h, const int32_t* d_tokens, const int32_t* d_targets, int B, int T, float* h_loss);
+/* Backward pass of the last forward-with-targets, scaling the loss by
+ * loss_scale (1/accumulation steps): every gradient += d(loss*loss_scale)/dparam
+ * ("Let's reproduce GPT-2 (124M)", Key Takeaways: gradient accumulation).
+ * The tied wte gradient receives both its lm_head and its embedding terms. */
+int gpt2_backward(gpt2_t* h, float loss_scale);
+/* Forward with targets and backward in one call, with the softmax gradient
+ * written in the same pass over the logits as the loss (the logits buffer is
+ * overwritten by its gradient, so gpt2_get_logits is unavailable after it). */
+int gpt2_forward_backward(gpt2_t* h, const int32_t* d_tokens, const int32_t* d_targets, int B, int T,
+                          float loss_scale, float* h_loss);
+/* Set every gradient to zero. */
+int gpt2_zero_grad(gpt2_t* h);
+/* Global-norm clip then AdamW ("Let's reproduce GPT-2 (124M)", Key Takeaways:
+ * optimization hyperparameters): n = ||g||_2 over all parameters (tied wte
+ * once), s = min(1, clip/(n + 1e-6)), g' = s*g; step t += 1;
+ * p *= 1 - lr*wd on 2D tensors (wte, wpe, Linear weights) only;
+ * m = b1 m + (1-b1) g'; v = b2 v + (1-b2) g'^2;
+ * p -= lr * (m/(1-b1^t)) / (sqrt(v/(1-b2^t)) + eps).
+ * A non-finite n leaves parameters, moments and t unchanged; it is reported
+ * as GPT2_ENONFINITE by this call when h_grad_norm is non-NULL (syncs) and
+ * otherwise by the next call that syncs.  h_grad_norm receives n. */
+int gpt2_adamw_step(gpt2_t* h, float lr, float wd, float b1, float b2, float eps, float clip, float* h_grad_norm);
+/* One whole optimizer step from HOST token buffers: zero_grad, then for each
+ * of n_micro micro-steps copy h_tokens/h_targets[k*B*T .. (k+1)*B*T) to the
+ * device and run forward+backward with loss_scale 1/n_micro, then
+ * gpt2_adamw_step.  h_loss receives the mean micro-step loss and h_grad_norm
+ * the pre-clip norm (both may be NULL; either one syncs). */
+int gpt2_train_step(gpt2_t* h, const int32_t* h_tokens, const int32_t* h_targets, int n_micro, int B, int T,
+                    float lr, float wd, float b1, float b2, float eps, float clip, float* h_loss,
+                    float* h_grad_norm);
+/* Learning rate at step `it`: linear warmup max_lr*(it+1)/warmup for it <
+ * warmup, min_lr after max_steps, cosine from max_lr to min_lr in between
+ * ("Let's reproduce GPT-2 (124M)", Chapters: learning rate scheduler; "From
+ * Scratch: Building GPT-2", Training Setup: 715 warmup steps, 19073 iterations). */
+double gpt2_lr_at(int it, double max_lr, double min_lr, int warmup, int max_steps);
+
+/* ---- accessors (parity checks, checkpoint / resume); all synchronise ---- */
+int64_t gpt2_num_params(const gpt2_t* h);
+int gpt2_get_params(gpt2_t* h, float* h_dst);       /* fp32 master weights, flat order */
+int gpt2_set_params(gpt2_t* h, const float* h_src); /* also refreshes the bf16 copy */
+int gpt2_get_grads(gpt2_t* h, float* h_dst);
+int gpt2_get_adam_state(gpt2_t* h, float* h_m, float* h_v, int64_t* h_step); /* any may be NULL */
+int gpt2_set_adam_state(gpt2_t* h, const float* h_m, const float* h_v, int64_t step);
+int gpt2_get_logits(gpt2_t* h, float* h_dst);  /* [B, T, Vp] of the last forward, as fp32 */
+int gpt2_get_argmax(gpt2_t* h, int32_t* h_dst); /* [B, T], lowest index among maxima */
+int gpt2_get_losses(gpt2_t* h, float* h_dst);   /* [B, T] per-position losses of the last forward */
+int gpt2_last_loss(gpt2_t* h, float* h_loss);   /* mean loss of the last forward with targets */
+/* Sorted (token << 16 | position) keys of the last backward's embedding
+ * scatter-add ([B*T] uint32, BF16 and FP32 modes). */
+int gpt2_get_embed_keys(gpt2_t* h, uint32_t* h_dst);
+/* Number of kernels this handle has launched since creation. */
+int64_t gpt2_kernel_launches(const gpt2_t* h);
+/* One-line description of the last failure on this handle (never NULL). */
+const char* gpt2_last_error(const gpt2_t* h);
+
+/* ---- standalone operators (device pointers, caller-owned memory) ---- */
+
+/* Causal multi-head attention forward, bf16, head dim 64, softmax scale
+ * 1/sqrt(64) ("Let's reproduce GPT-2 (124M)", Key Takeaways: architecture and
+ * flash attention bullets).  d_qkv: [B, T, 3C] bf16 with q, k, v the column
+ * blocks [0,C), [C,2C), [2C,3C) and head h in columns h*64..h*64+63 of each
+ * (C = 64*H).  d_out: [B, T, C] bf16.  d_lse: [B, H, T] fp32 natural-log
+ * softmax denominators.  Returns GPT2_EINVAL for non-positive sizes or
+ * pointers not 16-byte aligned. */
+int gpt2_attention_forward(const void* d_qkv, void* d_out, float* d_lse, int B, int T, int H, void* cuda_stream);
+/* Backward of gpt2_attention_forward: d_dqkv [B, T, 3C] bf16 receives dq, dk,
+ * dv in the same column layout.  d_work: caller-provided fp32 scratch of at
+ * least gpt2_attention_workspace_floats(B, T, H) elements (rowwise dO.O). */
+int gpt2_attention_backward(const void* d_qkv, const void* d_out, const void* d_dout, const float* d_lse,
+                            void* d_dqkv, float* d_work, int B, int T, int H, void* cuda_stream);
+int64_t gpt2_attention_workspace_floats(int B, int T, int H);
+
+/* bf16 tensor-core matrix product D[M,N] = sum_k A[m,k] B[n,k] (fp32
+ * accumulate) with a fused epilogue, the contraction every Linear layer of the
+ * model reduces to.  a_mn = 0: A stored [M][lda] (k contiguous), 1: [K][lda]
+ * (m contiguous); b_mn likewise for B ([N][ldb] or [K][ldb]).  epi:
+ *   0 out bf16 = D (+bias)          1 out fp32 = D (+bias)
+ *   2 out fp32 = resid + D (+bias)  3 out bf16 = u = D + bias, out2 bf16 = gelu_tanh(u)
+ *   4 out bf16 = D * gelu_tanh'(aux bf16)
+ *   5 out fp32 += D (split over K into d_work when d_work is non-NULL and large enough)
+ * out, resid, aux are [M][ldc].  lda, ldb, ldc multiples of 8; A, B, out
+ * 16-byte aligned.  bias: fp32 [N] or NULL.  GPT2_EINVAL otherwise. */
+int gpt2_matmul_bf16(const void* d_A, int64_t lda, int a_mn, const void* d_B, int64_t ldb, int b_mn, int M, int N,
+                     int K, int epi, const float* d_bias, const float* d_resid, void* d_out, void* d_out2,
+                     const void* d_aux, int64_t ldc, float* d_work, size_t work_bytes, void* cuda_stream);
+/* Bytes of d_work with which an epi = 5 call of this shape splits over K. */
+size_t gpt2_matmul_workspace_bytes(int M, int N, int K);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT2_B200_H */
