@@ -68,12 +68,12 @@ static int refresh_bf16(gpt2* h) {
 
 static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   std::string why;
+  if (validate_config(c, why) != GPT2_OK) return set_err(h, GPT2_EINVAL, why);
   {
     const cudaError_t stale = cudaGetLastError();
     if (stale != cudaSuccess)
       return set_err(h, GPT2_ECUDA, std::string("CUDA error pending before create: ") + cudaGetErrorString(stale));
   }
-  if (validate_config(c, why) != GPT2_OK) return set_err(h, GPT2_EINVAL, why);
   h->cfg = *c;
   h->L = c->n_layer;
   h->H = c->n_head;
