@@ -28,6 +28,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_t** out) {
 void gpt2_destroy(gpt2_t* h) {
   if (h == nullptr) return;
   cudaStreamSynchronize(h->stream);
+  for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   free_all(h);
   delete h;
 }
@@ -219,6 +220,34 @@ int gpt2_get_embed_keys(gpt2_t* h, uint32_t* dst) {
 }
 
 int64_t gpt2_kernel_launches(const gpt2_t* h) { return h ? h->launches : -1; }
+
+int gpt2_set_timing(gpt2_t* h, int enable) {
+  if (h == nullptr) return GPT2_EINVAL;
+  h->timing = enable != 0;
+  return GPT2_OK;
+}
+
+int gpt2_get_timing(gpt2_t* h, double* ms, int64_t* ops, double* flops, double* bytes) {
+  if (h == nullptr) return GPT2_EINVAL;
+  CU_CHECK(h, cudaStreamSynchronize(h->stream));
+  double t[GPT2_NUM_KCLASSES] = {};
+  int64_t n[GPT2_NUM_KCLASSES] = {};
+  for (size_t i = 0; i < h->ev_used; ++i) {
+    float e = 0.f;
+    CU_CHECK(h, cudaEventElapsedTime(&e, h->ev_pool[2 * i], h->ev_pool[2 * i + 1]));
+    t[h->ev_class[i]] += e;
+    n[h->ev_class[i]]++;
+  }
+  for (int c = 0; c < GPT2_NUM_KCLASSES; ++c) {
+    if (ms) ms[c] = t[c];
+    if (ops) ops[c] = n[c];
+    if (flops) flops[c] = h->t_flops[c];
+    if (bytes) bytes[c] = h->t_bytes[c];
+    h->t_flops[c] = h->t_bytes[c] = 0.0;
+  }
+  h->ev_used = 0;
+  return GPT2_OK;
+}
 
 const char* gpt2_last_error(const gpt2_t* h) { return h ? h->err.c_str() : g_null_handle_err.c_str(); }
 

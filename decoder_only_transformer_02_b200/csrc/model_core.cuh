@@ -79,6 +79,13 @@ struct gpt2 {
   const int32_t* last_tok = nullptr;
   const int32_t* last_tgt = nullptr;
 
+  // opt-in per-class device timing (measurement support)
+  bool timing = false;
+  std::vector<cudaEvent_t> ev_pool;   // 2 events per timed operation
+  std::vector<int> ev_class;          // class of each timed operation
+  size_t ev_used = 0;                 // operations recorded since the last read
+  double t_flops[GPT2_NUM_KCLASSES] = {}, t_bytes[GPT2_NUM_KCLASSES] = {};
+
   long M() const { return (long)B * T; }
   long Mmax() const { return (long)maxB * maxT; }
   float* P32(size_t off) { return params + off; }
@@ -195,3 +202,34 @@ static int colsum_rows_per_block(long M) {
   long r = (M + 127) / 128;
   return (int)(r < 16 ? 16 : r);
 }
+
+// Times one operation (all launches in its scope) when timing is enabled.
+struct KTimer {
+  gpt2* h;
+  int cls;
+  bool on;
+  KTimer(gpt2* hh, int c, double flops, double bytes) : h(hh), cls(c), on(hh->timing) {
+    if (!on) return;
+    if (h->ev_used * 2 + 2 > h->ev_pool.size()) {
+      for (int i = 0; i < 2; ++i) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) {
+          on = false;
+          return;
+        }
+        h->ev_pool.push_back(e);
+      }
+      h->ev_class.push_back(c);
+    }
+    h->ev_class[h->ev_used] = c;
+    cudaEventRecord(h->ev_pool[h->ev_used * 2], h->stream);
+    h->t_flops[c] += flops;
+    h->t_bytes[c] += bytes;
+  }
+  ~KTimer() {
+    if (!on) return;
+    cudaEventRecord(h->ev_pool[h->ev_used * 2 + 1], h->stream);
+    h->ev_used++;
+  }
+};
+enum KClass { KC_GEMM = 0, KC_ATTN_F, KC_ATTN_B, KC_LN_F, KC_LN_B, KC_CE, KC_OPT, KC_EMB, KC_OTHER };

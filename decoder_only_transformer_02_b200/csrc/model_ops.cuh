@@ -24,6 +24,7 @@ static int ln_fwd_dispatch(gpt2* h, const float* x, const float* g, const float*
 }
 
 static int op_ln_fwd(gpt2* h, const float* x, size_t goff, size_t boff, void* y, float* mean, float* rstd, long M) {
+  KTimer kt(h, KC_LN_F, 0.0, (double)M * h->C * (4 + h->es) + 8.0 * M);
   if (h->prec == GPT2_BF16)
     return ln_fwd_dispatch<bf16>(h, x, h->P32(goff), h->P32(boff), (bf16*)y, mean, rstd, M);
   return ln_fwd_dispatch<float>(h, x, h->P32(goff), h->P32(boff), (float*)y, mean, rstd, M);
@@ -34,6 +35,7 @@ static int op_ln_fwd(gpt2* h, const float* x, size_t goff, size_t boff, void* y,
 // the resulting residual gradient into the grads.
 static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean, const float* rstd, size_t goff,
                      size_t boff, size_t dbias_off, long M, int accumulate) {
+  KTimer kt(h, KC_LN_B, 0.0, (double)M * h->C * (12 + (accumulate ? 4 : 0) + (h->prec == GPT2_BF16 ? 2 : 0)) + 8.0 * M);
   const int rpb = ln_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
   bf16* dbf = h->prec == GPT2_BF16 ? h->dres_bf : nullptr;
@@ -74,6 +76,7 @@ static int simt_call(gpt2* h, const simt::Args& a) {
 // out[M,N] = X[M,K] W[N,K]^T (+ b): W at param offset woff, b at boff
 static int op_lin_fwd(gpt2* h, const void* X, long M, int K, size_t woff, int N, size_t boff, LinKind kind, void* out,
                       void* out2, const float* resid) {
+  KTimer kt(h, KC_GEMM, 2.0 * M * N * K, 0.0);
   const float* bias = boff == NO_OFF ? nullptr : h->P32(boff);
   if (h->prec == GPT2_BF16) {
     tcg::GemmArgs g;
@@ -124,6 +127,7 @@ enum DgradKind { DG_F32, DG_ACT, DG_DGELU };  // fp32 out / activation-typed out
 // dX[M,Kin] = dY[M,N] W[N,Kin]
 static int op_lin_dgrad(gpt2* h, const void* dY, long M, int N, size_t woff, int Kin, DgradKind kind, void* out,
                         const void* aux) {
+  KTimer kt(h, KC_GEMM, 2.0 * M * N * Kin, 0.0);
   if (h->prec == GPT2_BF16) {
     tcg::GemmArgs g;
     g.A = (const bf16*)dY;
@@ -160,6 +164,7 @@ static int op_lin_dgrad(gpt2* h, const void* dY, long M, int N, size_t woff, int
 
 // grads[W (N x Kin)] += dY[M,N]^T X[M,Kin]
 static int op_lin_wgrad(gpt2* h, const void* dY, long M, int N, const void* X, int Kin, size_t woff) {
+  KTimer kt(h, KC_GEMM, 2.0 * M * N * Kin, 0.0);
   if (h->prec == GPT2_BF16) {
     tcg::GemmArgs g;
     g.A = (const bf16*)dY;
@@ -196,6 +201,7 @@ static int op_lin_wgrad(gpt2* h, const void* dY, long M, int N, const void* X, i
 
 // grads[boff .. +N] += column sums of a[M, N] (activation type)
 static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
+  KTimer kt(h, KC_OTHER, 0.0, (double)M * N * h->es);
   const int rpb = colsum_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
   dim3 grid((N + 255) / 256, nblk);
@@ -211,6 +217,7 @@ static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
 
 // --------------------------------------------------------------- attention
 static int op_attn_fwd(gpt2* h, int l) {
+  KTimer kt(h, KC_ATTN_F, 2.0 * h->B * (double)h->T * h->T * h->C, 0.0);
   const long M = h->M();
   uint8_t* qkv = h->qkv + (size_t)l * h->Mmax() * 3 * h->C * h->es;
   uint8_t* att = h->att + (size_t)l * h->Mmax() * h->C * h->es;
@@ -230,6 +237,7 @@ static int op_attn_fwd(gpt2* h, int l) {
 }
 
 static int op_attn_bwd(gpt2* h, int l) {
+  KTimer kt(h, KC_ATTN_B, 4.0 * h->B * (double)h->T * h->T * h->C, 0.0);
   uint8_t* qkv = h->qkv + (size_t)l * h->Mmax() * 3 * h->C * h->es;
   uint8_t* att = h->att + (size_t)l * h->Mmax() * h->C * h->es;
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;

@@ -42,9 +42,12 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
     CU_CHECK(h, cudaMemcpyAsync(h->tgt_dev, tgt, M * 4, cudaMemcpyDeviceToDevice, h->stream));
   const int32_t* dtgt = tgt ? h->tgt_dev : nullptr;
 
-  k::embed_fwd_kernel<<<grid_for(M * C / 4, 256), 256, 0, h->stream>>>(h->tok_dev, dtgt, h->P32(h->wte), h->P32(h->wpe),
-                                                                      w.res(0), (int)M, T, C, h->Vp, h->d_bad);
-  LAUNCH_CHECK(h);
+  {
+    KTimer kt(h, KC_EMB, 0.0, 12.0 * M * C);
+    k::embed_fwd_kernel<<<grid_for(M * C / 4, 256), 256, 0, h->stream>>>(
+        h->tok_dev, dtgt, h->P32(h->wte), h->P32(h->wpe), w.res(0), (int)M, T, C, h->Vp, h->d_bad);
+    LAUNCH_CHECK(h);
+  }
   for (int l = 0; l < L; ++l) {
     const LayerOffsets& o = h->lo[l];
     RET_IF(op_ln_fwd(h, w.res(2 * l), o.ln1g, o.ln1b, w.ln1(l), w.ln1m(l), w.ln1r(l), M));
@@ -61,6 +64,8 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
   RET_IF(op_lin_fwd(h, h->lnf, M, C, h->wte, h->Vp, NO_OFF, LIN_NOBIAS, h->logits, nullptr, nullptr));
   const size_t smem = (size_t)h->Vp * h->es;
   const float gscale = loss_scale / (float)M;
+  {
+  KTimer kt(h, KC_CE, 0.0, (double)M * h->Vp * h->es * (fuse ? 2 : 1));
   if (h->prec == GPT2_BF16)
     k::ce_kernel<bf16><<<(unsigned)M, 1024, smem, h->stream>>>((bf16*)h->logits, dtgt, h->Vp, h->ce_lse,
                                                                 dtgt ? h->losses : nullptr, h->argmax, fuse ? 1 : 0,
@@ -70,7 +75,9 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
                                                                  dtgt ? h->losses : nullptr, h->argmax, fuse ? 1 : 0,
                                                                  gscale);
   LAUNCH_CHECK(h);
+  }
   if (dtgt) {
+    KTimer kt(h, KC_OTHER, 0.0, 4.0 * M);
     k::loss_mean_kernel<<<1, 1024, 0, h->stream>>>(h->losses, (int)M, h->d_loss, h->d_loss + 1,
                                                    fuse ? loss_scale : 0.f);
     LAUNCH_CHECK(h);
@@ -89,6 +96,7 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
   const int C = h->C, L = h->L, B = h->B, T = h->T;
   Views w{h};
   if (!fused) {
+    KTimer kt(h, KC_CE, 0.0, 2.0 * M * h->Vp * h->es);
     const float gscale = loss_scale / (float)M;
     if (h->prec == GPT2_BF16)
       k::ce_bwd_kernel<bf16><<<(unsigned)M, 512, 0, h->stream>>>((bf16*)h->logits, h->tgt_dev, h->ce_lse, h->Vp,
@@ -126,6 +134,7 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
                      M, 1));
   }
   // embeddings: dwte[tok] += dx0 (sorted, fixed order), dwpe[t] += sum_b dx0[b, t]
+  KTimer kt(h, KC_EMB, 0.0, 8.0 * M * C + 8.0 * T * C);
   k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->stream>>>(h->tok_dev, (int)M, h->Vp, h->emb_keys,
                                                                         h->sort_cap);
   LAUNCH_CHECK(h);
@@ -145,6 +154,7 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
 
 static int adamw_impl(gpt2* h, float lr, float wd, float b1, float b2, float eps, float clip) {
   const long n = (long)h->nparams;
+  KTimer kt(h, KC_OPT, 0.0, 34.0 * n);
   long per = (n + h->norm_blocks - 1) / h->norm_blocks;
   per = (per + 3) / 4 * 4;
   k::sumsq_partial_kernel<<<h->norm_blocks, 256, 0, h->stream>>>(h->grads, n, per, h->norm_part);

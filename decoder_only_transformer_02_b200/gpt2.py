@@ -26,8 +26,10 @@ EXPORTED = [
     "gpt2_set_params", "gpt2_get_grads", "gpt2_get_adam_state", "gpt2_set_adam_state", "gpt2_get_logits",
     "gpt2_get_argmax", "gpt2_get_losses", "gpt2_last_loss", "gpt2_get_embed_keys", "gpt2_kernel_launches",
     "gpt2_last_error", "gpt2_attention_forward", "gpt2_attention_backward", "gpt2_attention_workspace_floats",
-    "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes",
+    "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes", "gpt2_set_timing", "gpt2_get_timing",
 ]
+KCLASSES = ["matmul", "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd", "cross_entropy",
+            "optimizer", "embedding", "other"]
 
 
 class GPT2Error(RuntimeError):
@@ -84,6 +86,8 @@ def load_library():
         "gpt2_attention_workspace_floats": (L, [I, I, I]),
         "gpt2_matmul_bf16": (I, [P, L, I, P, L, I, I, I, I, I, P, P, P, P, P, L, P, S, P]),
         "gpt2_matmul_workspace_bytes": (S, [I, I, I]),
+        "gpt2_set_timing": (I, [P, I]),
+        "gpt2_get_timing": (I, [P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -202,6 +206,23 @@ class GPT2:
                                               b1, b2, eps, clip, ctypes.byref(loss) if want else None,
                                               ctypes.byref(norm) if want else None))
         return (loss.value, norm.value) if want else None
+
+    # -- measurement support
+    def set_timing(self, enable: bool):
+        self._check(self._lib.gpt2_set_timing(self._h, 1 if enable else 0))
+
+    def get_timing(self) -> dict:
+        """Per kernel class: device ms, operations, algorithmic FLOPs and bytes
+        since the last call (then reset)."""
+        n = len(KCLASSES)
+        ms = np.zeros(n, dtype=np.float64)
+        ops = np.zeros(n, dtype=np.int64)
+        fl = np.zeros(n, dtype=np.float64)
+        by = np.zeros(n, dtype=np.float64)
+        self._check(self._lib.gpt2_get_timing(self._h, ms.ctypes.data, ops.ctypes.data, fl.ctypes.data,
+                                              by.ctypes.data))
+        return {k: dict(ms=float(ms[i]), ops=int(ops[i]), flops=float(fl[i]), bytes=float(by[i]))
+                for i, k in enumerate(KCLASSES)}
 
     # -- accessors
     @property

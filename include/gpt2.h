@@ -137,6 +137,23 @@ int gpt2_last_loss(gpt2_t* h, float* h_loss);   /* mean loss of the last forward
 int gpt2_get_embed_keys(gpt2_t* h, uint32_t* h_dst);
 /* Number of kernels this handle has launched since creation. */
 int64_t gpt2_kernel_launches(const gpt2_t* h);
+
+/* ---- measurement support ----
+ * With timing enabled, every operation this handle enqueues is bracketed by a
+ * pair of CUDA events on the handle's stream and its device time is
+ * accumulated per kernel class, together with the operation's algorithmic
+ * work: FLOPs (2*M*N*K for a matrix product, 4*B*H*d*(causal score count) for
+ * attention forward, twice that for its backward) and the bytes an ideal
+ * kernel must move through HBM.  Classes (array index):
+ *   0 matmul (tcgen05 GEMM and its split-K reduction)  1 attention forward
+ *   2 attention backward  3 LayerNorm forward  4 LayerNorm backward (+ bias sums)
+ *   5 cross-entropy  6 gradient norm + AdamW  7 embedding  8 other (colsum, loss mean) */
+#define GPT2_NUM_KCLASSES 9
+int gpt2_set_timing(gpt2_t* h, int enable);
+/* Synchronise, then fill h_ms / h_ops / h_flops / h_bytes (arrays of
+ * GPT2_NUM_KCLASSES; any may be NULL) with the totals since the last call, and
+ * reset them.  h_ops counts timed operations (one or two kernels each). */
+int gpt2_get_timing(gpt2_t* h, double* h_ms, int64_t* h_ops, double* h_flops, double* h_bytes);
 /* One-line description of the last failure on this handle (never NULL). */
 const char* gpt2_last_error(const gpt2_t* h);
 
