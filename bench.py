@@ -325,8 +325,74 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------- standalone operators
+
+def run_op(args):
+    """One operator of the step alone, timed with CUDA events (burst peak).
+    matmul: D[M,N] = A B^T in the forward / dgrad / wgrad layout of the model.
+    attention: causal fwd+bwd, B=8, H=12, d=64 (the standalone attention workload)."""
+    import torch
+    from decoder_only_transformer_02_b200 import gpt2 as G
+    from decoder_only_transformer_02_b200.synthetic import normal_array
+    torch.cuda.set_device(0)
+    peaks, kind = load_peaks()
+    st = torch.cuda.current_stream()
+    out = {"op": args.op, "peak_source": kind}
+    if args.op == "matmul":
+        M, N, K = (int(x) for x in args.shape.split(","))
+        a_mn, b_mn = {"fwd": (0, 0), "dgrad": (0, 1), "wgrad": (1, 1)}[args.layout]
+        A = torch.from_numpy(normal_array((K, M) if a_mn else (M, K), 1)).to(torch.bfloat16).cuda()
+        Bm = torch.from_numpy(normal_array((K, N) if b_mn else (N, K), 2)).to(torch.bfloat16).cuda()
+        epi = 5 if args.layout == "wgrad" else 0
+        o = torch.zeros(M, N, dtype=torch.float32 if epi == 5 else torch.bfloat16, device="cuda")
+        wsb = G.matmul_workspace_bytes(M, N, K) if epi == 5 else 0
+        ws = torch.empty(max(1, wsb // 4), dtype=torch.float32, device="cuda")
+        call = lambda: G.matmul_bf16(A, M if a_mn else K, a_mn, Bm, N if b_mn else K, b_mn, M, N, K, epi, out=o,
+                                     ldc=N, work=ws if wsb else None, work_bytes=wsb, stream=st)
+        work = 2.0 * M * N * K
+        out.update(shape=[M, N, K], layout=args.layout, splitk_workspace_bytes=wsb)
+    else:
+        B, H, T = 8, 12, args.T
+        Cc = 64 * H
+        qkv = torch.from_numpy(normal_array((B, T, 3 * Cc), 3)).to(torch.bfloat16).cuda()
+        do = torch.from_numpy(normal_array((B, T, Cc), 4)).to(torch.bfloat16).cuda()
+        o = torch.empty(B, T, Cc, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+        dqkv = torch.empty_like(qkv)
+        wk = torch.empty(G.attention_workspace_floats(B, T, H), dtype=torch.float32, device="cuda")
+        fwd = lambda: G.attention_forward(qkv, o, lse, B, T, H, stream=st)
+        bwd = lambda: G.attention_backward(qkv, o, do, lse, dqkv, wk, B, T, H, stream=st)
+        if args.part == "fwd":
+            call, work = fwd, 2.0 * B * H * T * T * 64
+        elif args.part == "bwd":
+            fwd()
+            call, work = bwd, 4.0 * B * H * T * T * 64
+        else:
+            call, work = (lambda: (fwd(), bwd())), 6.0 * B * H * T * T * 64
+        out.update(B=B, H=H, T=T, d=64, part=args.part, flops_convention="causal: fwd 2*B*H*T^2*d, bwd 2x fwd")
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        call()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    tf = work / (ms / 1e3) / 1e12
+    out.update(ms_per_call=ms, tflops=tf, peak_bf16_tflops=peaks["bf16_tflops"], frac=tf / peaks["bf16_tflops"])
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--op", choices=["matmul", "attention"], default=None)
+    ap.add_argument("--shape", default="16384,3072,768")
+    ap.add_argument("--layout", choices=["fwd", "dgrad", "wgrad"], default="fwd")
+    ap.add_argument("--T", type=int, default=1024)
+    ap.add_argument("--part", choices=["fwd", "bwd", "both"], default="both")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
@@ -334,6 +400,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="t1024")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.op:
+        return run_op(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
