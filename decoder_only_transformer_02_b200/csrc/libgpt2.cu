@@ -4,8 +4,33 @@
 #include "tc_gemm.cu"
 #include "model_pass.cuh"
 
+#include <mutex>
+
 
 static std::string g_null_handle_err = "handle is NULL";
+
+// Scratch of gpt2_attention_backward_noalloc: a fixed device array (one fp32
+// per attention row), so that entry point never allocates.  Host code cannot
+// use the symbol itself as a device address: the address is looked up once per
+// device, with that device current, and cached.
+static __device__ __align__(256) float g_attn_noalloc_scratch[GPT2_ATTN_NOALLOC_MAX_ROWS];
+static std::mutex g_noalloc_mu;
+static float* g_noalloc_addr[256] = {};
+
+static float* noalloc_scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  return g_noalloc_addr[dev];
+}
 
 extern "C" {
 
@@ -304,5 +329,18 @@ int gpt2_matmul_bf16(const void* A, int64_t lda, int a_mn, const void* Bm, int64
 }
 
 size_t gpt2_matmul_workspace_bytes(int M, int N, int K) { return tcg::splitk_workspace_bytes(M, N, K, 0); }
+
+int gpt2_attention_backward_noalloc(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv,
+                                    int B, int T, int H, void* stream) {
+  if (!qkv || !out || !dout || !lse || !dqkv || B < 1 || T < 1 || H < 1) return GPT2_EINVAL;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(dqkv)) return GPT2_EINVAL;
+  if ((long long)B * H * T > (long long)GPT2_ATTN_NOALLOC_MAX_ROWS) return GPT2_EINVAL;
+  float* scratch = noalloc_scratch_on_current_device();
+  if (scratch == nullptr) return GPT2_ECUDA;
+  return attn::flash_backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, scratch, B, T,
+                              H, (cudaStream_t)stream) == cudaSuccess
+             ? GPT2_OK
+             : GPT2_ECUDA;
+}
 
 }  // extern "C"

@@ -27,7 +27,9 @@ EXPORTED = [
     "gpt2_get_argmax", "gpt2_get_losses", "gpt2_last_loss", "gpt2_get_embed_keys", "gpt2_kernel_launches",
     "gpt2_last_error", "gpt2_attention_forward", "gpt2_attention_backward", "gpt2_attention_workspace_floats",
     "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes", "gpt2_set_timing", "gpt2_get_timing",
+    "gpt2_attention_backward_noalloc",
 ]
+ATTN_NOALLOC_MAX_ROWS = 1 << 20
 KCLASSES = ["matmul", "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd", "cross_entropy",
             "optimizer", "embedding", "other"]
 
@@ -88,6 +90,7 @@ def load_library():
         "gpt2_matmul_workspace_bytes": (S, [I, I, I]),
         "gpt2_set_timing": (I, [P, I]),
         "gpt2_get_timing": (I, [P, P, P, P, P]),
+        "gpt2_attention_backward_noalloc": (I, [P, P, P, P, P, I, I, I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -306,6 +309,14 @@ def attention_backward(qkv, out, dout, lse, dqkv, work, B, T, H, stream=None):
     _op_check(load_library().gpt2_attention_backward(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv),
                                                      _ptr(work), B, T, H, _stream_ptr(stream)),
               "gpt2_attention_backward")
+
+
+def attention_backward_noalloc(qkv, out, dout, lse, dqkv, B, T, H, stream=None):
+    """gpt2_attention_backward with the library's fixed scratch array (no
+    allocation; B*H*T <= ATTN_NOALLOC_MAX_ROWS; calls must not overlap)."""
+    _op_check(load_library().gpt2_attention_backward_noalloc(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse),
+                                                             _ptr(dqkv), B, T, H, _stream_ptr(stream)),
+              "gpt2_attention_backward_noalloc")
 
 
 def matmul_bf16(A, lda, a_mn, Bm, ldb, b_mn, M, N, K, epi, bias=None, resid=None, out=None, out2=None, aux=None,

@@ -190,6 +190,29 @@ int gpt2_matmul_bf16(const void* d_A, int64_t lda, int a_mn, const void* d_B, in
 /* Bytes of d_work with which an epi = 5 call of this shape splits over K. */
 size_t gpt2_matmul_workspace_bytes(int M, int N, int K);
 
+/* ---- attention backward without any allocation ----
+ * (No counterpart in the paper: this is a calling convenience of this library.)
+ * The same computation as gpt2_attention_backward, for callers that cannot
+ * call cudaMalloc and have no spare device buffer to hand over as d_work: for
+ * example a host framework that plans every byte of device memory ahead of
+ * time and forbids allocations outside its planner, or a process that runs
+ * with the device memory already fully reserved.  Its scratch (one fp32 per
+ * (batch, head, position) row) lives in a fixed array inside the library, of
+ * GPT2_ATTN_NOALLOC_MAX_ROWS floats (4 MiB); every GPU that loads the library
+ * holds that array until the process exits.
+ *  - B*H*T must be at most GPT2_ATTN_NOALLOC_MAX_ROWS, else GPT2_EINVAL and
+ *    nothing is enqueued.  Other arguments as for gpt2_attention_backward.
+ *  - The first call on each device looks up the array's device address on
+ *    that device (with it current); make that first call before any stream
+ *    capture.  No call allocates device or host memory.
+ *  - All calls share the one array and it keeps the last call's contents; the
+ *    kernel overwrites every scratch element it reads, so nothing needs to be
+ *    cleared.  Calls that overlap on the GPU (different streams, or different
+ *    host threads on one device) race on the array: serialise them. */
+#define GPT2_ATTN_NOALLOC_MAX_ROWS (1 << 20)
+int gpt2_attention_backward_noalloc(const void* d_qkv, const void* d_out, const void* d_dout, const float* d_lse,
+                                    void* d_dqkv, int B, int T, int H, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
