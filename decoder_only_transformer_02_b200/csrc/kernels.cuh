@@ -193,140 +193,160 @@ __global__ void ln_fwd_kernel(const float* __restrict__ x, const float* __restri
 // LayerNorm backward fused with the residual stream.  One warp per row:
 //   dxhat = dy*g ; dx = rstd*(dxhat - mean(dxhat) - xhat*mean(dxhat*xhat))
 //   dres = (accumulate ? dres : 0) + dx     (fp32, in place)   and a bf16 copy
-// Per-block partial column sums (fixed row ranges, fixed order) of
+// and per-block partial column sums (fixed row ranges, fixed order) of
 //   dy*xhat (-> dgamma), dy (-> dbeta), dres_out (-> the bias gradient of the
 //   linear layer whose output is this residual point).
+// The column accumulators live in shared memory, one private slice per warp
+// (each lane owns its columns: no conflicts, no atomics), which keeps the
+// register count low enough for several CTAs per SM; all loads of a row are
+// issued before its reductions.  Dynamic shared memory: 3 * C * LN_BWD_WARPS floats.
+constexpr int LN_BWD_WARPS = 4;
 template <int NV, typename TI>
-__global__ void __launch_bounds__(256) ln_bwd_kernel(const TI* __restrict__ dy, const float* __restrict__ x,
+__global__ void __launch_bounds__(LN_BWD_WARPS * 32, 3) ln_bwd_kernel(const TI* __restrict__ dy, const float* __restrict__ x,
                                                      const float* __restrict__ mean, const float* __restrict__ rstd,
                                                      const float* __restrict__ gam, float* __restrict__ dres,
                                                      bf16* __restrict__ dres_bf, int M, int rows_per_block,
                                                      int accumulate, float* __restrict__ part) {
   constexpr int C = 128 * NV;
-  constexpr int WARPS = 8;
-  __shared__ float4 red[3 * C / 4];
+  constexpr int C4 = C / 4;
+  extern __shared__ float4 ln_acc[];  // [warp][3][C4]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float4 pg[NV], pb[NV], pd[NV];
+  float4* acc = ln_acc + warp * 3 * C4;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) pg[i] = pb[i] = pd[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 gv[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) gv[i] = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
+  for (int i = 0; i < NV; ++i) {
+    const int c4 = lane + 32 * i;
+    acc[c4] = acc[C4 + c4] = acc[2 * C4 + c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const long r0 = (long)blockIdx.x * rows_per_block;
   const long r1 = min((long)M, r0 + rows_per_block);
-  for (long row = r0 + warp; row < r1; row += WARPS) {
+  for (long row = r0 + warp; row < r1; row += LN_BWD_WARPS) {
     const float mu = mean[row], rs = rstd[row];
-    float4 xh[NV], dyv[NV];
+    const float4* xr = reinterpret_cast<const float4*>(x + row * C) + lane;
+    float4* dr = reinterpret_cast<float4*>(dres + row * C) + lane;
+    float4 xv[NV], dyv[NV], rv[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      xv[i] = xr[32 * i];
+      if constexpr (sizeof(TI) == 2) {
+        const uint2 u = reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(dy) + row * C)[lane + 32 * i];
+        const float2 a0 = unpack_bf16x2(u.x), a1 = unpack_bf16x2(u.y);
+        dyv[i] = make_float4(a0.x, a0.y, a1.x, a1.y);
+      } else {
+        dyv[i] = (reinterpret_cast<const float4*>(reinterpret_cast<const float*>(dy) + row * C) + lane)[32 * i];
+      }
+      rv[i] = accumulate ? dr[32 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      const int c = 4 * (lane + 32 * i);
-      const float4 xv = *reinterpret_cast<const float4*>(x + row * C + c);
-      xh[i] = make_float4((xv.x - mu) * rs, (xv.y - mu) * rs, (xv.z - mu) * rs, (xv.w - mu) * rs);
-      if constexpr (sizeof(TI) == 2) {
-        const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(dy) + row * C + c);
-        const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
-        dyv[i] = make_float4(a.x, a.y, b.x, b.y);
-      } else {
-        dyv[i] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(dy) + row * C + c);
-      }
-      const float d0 = dyv[i].x * gv[i].x, d1 = dyv[i].y * gv[i].y, d2 = dyv[i].z * gv[i].z, d3 = dyv[i].w * gv[i].w;
+      const float4 g = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
+      xv[i] = make_float4((xv[i].x - mu) * rs, (xv[i].y - mu) * rs, (xv[i].z - mu) * rs, (xv[i].w - mu) * rs);
+      const float d0 = dyv[i].x * g.x, d1 = dyv[i].y * g.y, d2 = dyv[i].z * g.z, d3 = dyv[i].w * g.w;
       s1 += d0 + d1 + d2 + d3;
-      s2 += d0 * xh[i].x + d1 * xh[i].y + d2 * xh[i].z + d3 * xh[i].w;
+      s2 += d0 * xv[i].x + d1 * xv[i].y + d2 * xv[i].z + d3 * xv[i].w;
     }
     s1 = warp_sum(s1) * (1.f / C);
     s2 = warp_sum(s2) * (1.f / C);
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      const int c = 4 * (lane + 32 * i);
+      const int c4 = lane + 32 * i;
+      const float4 g = reinterpret_cast<const float4*>(gam)[c4];
       float4 o;
-      o.x = rs * (dyv[i].x * gv[i].x - s1 - xh[i].x * s2);
-      o.y = rs * (dyv[i].y * gv[i].y - s1 - xh[i].y * s2);
-      o.z = rs * (dyv[i].z * gv[i].z - s1 - xh[i].z * s2);
-      o.w = rs * (dyv[i].w * gv[i].w - s1 - xh[i].w * s2);
-      float4* dp = reinterpret_cast<float4*>(dres + row * C + c);
-      if (accumulate) {
-        const float4 r = *dp;
-        o.x += r.x;
-        o.y += r.y;
-        o.z += r.z;
-        o.w += r.w;
-      }
-      *dp = o;
+      o.x = rv[i].x + rs * (dyv[i].x * g.x - s1 - xv[i].x * s2);
+      o.y = rv[i].y + rs * (dyv[i].y * g.y - s1 - xv[i].y * s2);
+      o.z = rv[i].z + rs * (dyv[i].z * g.z - s1 - xv[i].z * s2);
+      o.w = rv[i].w + rs * (dyv[i].w * g.w - s1 - xv[i].w * s2);
+      dr[32 * i] = o;
       if (dres_bf != nullptr)
-        *reinterpret_cast<uint2*>(dres_bf + row * C + c) = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
-      pg[i].x += dyv[i].x * xh[i].x;
-      pg[i].y += dyv[i].y * xh[i].y;
-      pg[i].z += dyv[i].z * xh[i].z;
-      pg[i].w += dyv[i].w * xh[i].w;
-      pb[i].x += dyv[i].x;
-      pb[i].y += dyv[i].y;
-      pb[i].z += dyv[i].z;
-      pb[i].w += dyv[i].w;
-      pd[i].x += o.x;
-      pd[i].y += o.y;
-      pd[i].z += o.z;
-      pd[i].w += o.w;
+        reinterpret_cast<uint2*>(dres_bf + row * C)[c4] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+      float4 a = acc[c4], b = acc[C4 + c4], d = acc[2 * C4 + c4];
+      a.x += dyv[i].x * xv[i].x;
+      a.y += dyv[i].y * xv[i].y;
+      a.z += dyv[i].z * xv[i].z;
+      a.w += dyv[i].w * xv[i].w;
+      b.x += dyv[i].x;
+      b.y += dyv[i].y;
+      b.z += dyv[i].z;
+      b.w += dyv[i].w;
+      d.x += o.x;
+      d.y += o.y;
+      d.z += o.z;
+      d.w += o.w;
+      acc[c4] = a;
+      acc[C4 + c4] = b;
+      acc[2 * C4 + c4] = d;
     }
   }
-  // block reduction over warps, in warp order
-  for (int w = 0; w < WARPS; ++w) {
-    if (warp == w) {
+  __syncthreads();
+  // combine the warps' slices in warp order
+  const float* af = reinterpret_cast<const float*>(ln_acc);
+  for (int idx = threadIdx.x; idx < 3 * C; idx += blockDim.x) {
+    float t = 0.f;
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int c4 = lane + 32 * i;
-        float4 a = pg[i], b = pb[i], d = pd[i];
-        if (w > 0) {
-          const float4 ra = red[c4], rb = red[C / 4 + c4], rd = red[2 * (C / 4) + c4];
-          a = make_float4(ra.x + a.x, ra.y + a.y, ra.z + a.z, ra.w + a.w);
-          b = make_float4(rb.x + b.x, rb.y + b.y, rb.z + b.z, rb.w + b.w);
-          d = make_float4(rd.x + d.x, rd.y + d.y, rd.z + d.z, rd.w + d.w);
-        }
-        red[c4] = a;
-        red[C / 4 + c4] = b;
-        red[2 * (C / 4) + c4] = d;
-      }
-    }
-    __syncthreads();
-  }
-  const float* rf = reinterpret_cast<const float*>(red);
-  for (int idx = threadIdx.x; idx < 3 * C; idx += blockDim.x) part[(long)blockIdx.x * 3 * C + idx] = rf[idx];
-}
-
-// sum the per-block partials (fixed order) into dgamma, dbeta and, when given,
-// a bias gradient: out_k[c] += sum_blk part[blk][k][c]
-__global__ void ln_bwd_finish_kernel(const float* __restrict__ part, int nblk, int C, float* __restrict__ dg,
-                                     float* __restrict__ db, float* __restrict__ dbias) {
-  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < 3 * C; idx += gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int b = 0; b < nblk; ++b) acc += part[(long)b * 3 * C + idx];
-    const int which = idx / C, c = idx % C;
-    if (which == 0)
-      dg[c] += acc;
-    else if (which == 1)
-      db[c] += acc;
-    else if (dbias != nullptr)
-      dbias[c] += acc;
+    for (int w = 0; w < LN_BWD_WARPS; ++w) t += af[w * 3 * C + idx];
+    part[(long)blockIdx.x * 3 * C + idx] = t;
   }
 }
 
-// column sums of an [M, N] matrix into out[N] (+=), two stages, fixed order
+// Sum per-block partial rows (fixed order) into up to three outputs:
+// part is [nblk][ncols]; column j goes to out[j / C][j % C] (+=).  One warp
+// per 32 columns and block; the 8 warps of a block take every 8th partial row
+// and are combined in warp order, so the result is independent of timing.
+__global__ void __launch_bounds__(256) partials_reduce_kernel(const float* __restrict__ part, int nblk, int ncols, int C,
+                                                              float* __restrict__ out0, float* __restrict__ out1,
+                                                              float* __restrict__ out2) {
+  __shared__ float red[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int col = blockIdx.x * 32 + lane;
+  float s = 0.f;
+  if (col < ncols)
+    for (int b = warp; b < nblk; b += 8) s += part[(long)b * ncols + col];
+  red[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && col < ncols) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    const int which = col / C, c = col % C;
+    float* o = which == 0 ? out0 : (which == 1 ? out1 : out2);
+    if (o != nullptr) o[c] += t;
+  }
+}
+
+// Column sums of an [M, N] matrix, stage 1: block (x, y) sums 32 column
+// groups of 16 bytes (8 bf16 or 4 fp32 columns each) over rows
+// [y*rows_per_block, ...), 8 row lanes per group, combined in lane order.
+// N must be a multiple of 16 / sizeof(T).
 template <typename T>
-__global__ void colsum_partial_kernel(const T* __restrict__ a, int M, int N, int rows_per_block,
-                                      float* __restrict__ part) {
+__global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ a, int M, int N, int rows_per_block,
+                                                             float* __restrict__ part) {
+  constexpr int VEC = 16 / sizeof(T);
+  __shared__ float red[8][32 * VEC];
+  const int cg = threadIdx.x & 31, rl = threadIdx.x >> 5;
+  const int c0 = (blockIdx.x * 32 + cg) * VEC;
   const int r0 = blockIdx.y * rows_per_block;
   const int r1 = min(M, r0 + rows_per_block);
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < N; c += gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int r = r0; r < r1; ++r) acc += ld_f(a + (long)r * N + c);
-    part[(long)blockIdx.y * N + c] = acc;
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+  if (c0 < N) {
+#pragma unroll 4
+    for (int r = r0 + rl; r < r1; r += 8) {
+      const uint4 u = *reinterpret_cast<const uint4*>(a + (long)r * N + c0);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] += ld_f(e + i);
+    }
   }
-}
-__global__ void colsum_finish_kernel(const float* __restrict__ part, int nblk, int N, float* __restrict__ out) {
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < N; c += gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int b = 0; b < nblk; ++b) acc += part[(long)b * N + c];
-    out[c] += acc;
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) red[rl][cg * VEC + i] = acc[i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < 32 * VEC; i += 256) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][i];
+    const int col = blockIdx.x * 32 * VEC + i;
+    if (col < N) part[(long)blockIdx.y * N + col] = t;
   }
 }
 

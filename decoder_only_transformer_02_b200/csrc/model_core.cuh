@@ -192,15 +192,16 @@ static void free_all(gpt2* h) {
     if (p) cudaFree(p);
 }
 
-// rows handled per CTA by the LayerNorm backward (multiple of 8 warps)
+// rows handled per CTA by the LayerNorm backward: about 4 CTAs per SM
 static int ln_rows_per_block(long M) {
-  long r = (M + 295) / 296;
-  r = (r + 7) / 8 * 8;
-  return (int)(r < 8 ? 8 : r);
+  long r = (M + 591) / 592;
+  r = (r + 3) / 4 * 4;
+  return (int)(r < 4 ? 4 : r);
 }
+// rows per CTA of the column-sum kernel: at most 64 row blocks
 static int colsum_rows_per_block(long M) {
-  long r = (M + 127) / 128;
-  return (int)(r < 16 ? 16 : r);
+  long r = (M + 63) / 64;
+  return (int)(r < 64 ? 64 : r);
 }
 
 // Times one operation (all launches in its scope) when timing is enabled.

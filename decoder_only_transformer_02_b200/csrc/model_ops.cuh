@@ -39,11 +39,12 @@ static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean
   const int rpb = ln_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
   bf16* dbf = h->prec == GPT2_BF16 ? h->dres_bf : nullptr;
+  const size_t smem = (size_t)3 * h->C * k::LN_BWD_WARPS * sizeof(float);
   switch (h->C / 128) {
 #define LNB(NV)                                                                                                     \
   case NV:                                                                                                          \
-    k::ln_bwd_kernel<NV, float><<<nblk, 256, 0, h->stream>>>(dy, x, mean, rstd, h->P32(goff), h->dres, dbf, (int)M, \
-                                                             rpb, accumulate, h->ln_part);                          \
+    k::ln_bwd_kernel<NV, float><<<nblk, k::LN_BWD_WARPS * 32, smem, h->stream>>>(                                 \
+        dy, x, mean, rstd, h->P32(goff), h->dres, dbf, (int)M, rpb, accumulate, h->ln_part);                        \
     break;
     LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
 #undef LNB
@@ -51,8 +52,9 @@ static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean
       return set_err(h, GPT2_EINVAL, "n_embd must be a multiple of 128 up to 1024");
   }
   LAUNCH_CHECK(h);
-  k::ln_bwd_finish_kernel<<<grid_for(3 * h->C, 256), 256, 0, h->stream>>>(
-      h->ln_part, nblk, h->C, h->G32(goff), h->G32(boff), dbias_off == NO_OFF ? nullptr : h->G32(dbias_off));
+  k::partials_reduce_kernel<<<(3 * h->C + 31) / 32, 256, 0, h->stream>>>(
+      h->ln_part, nblk, 3 * h->C, h->C, h->G32(goff), h->G32(boff),
+      dbias_off == NO_OFF ? nullptr : h->G32(dbias_off));
   LAUNCH_CHECK(h);
   return GPT2_OK;
 }
@@ -204,13 +206,15 @@ static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
   KTimer kt(h, KC_OTHER, 0.0, (double)M * N * h->es);
   const int rpb = colsum_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
-  dim3 grid((N + 255) / 256, nblk);
+  const int vec = h->prec == GPT2_BF16 ? 8 : 4;
+  dim3 grid((N + 32 * vec - 1) / (32 * vec), nblk);
   if (h->prec == GPT2_BF16)
     k::colsum_partial_kernel<bf16><<<grid, 256, 0, h->stream>>>((const bf16*)a, (int)M, N, rpb, h->cs_part);
   else
     k::colsum_partial_kernel<float><<<grid, 256, 0, h->stream>>>((const float*)a, (int)M, N, rpb, h->cs_part);
   LAUNCH_CHECK(h);
-  k::colsum_finish_kernel<<<(N + 255) / 256, 256, 0, h->stream>>>(h->cs_part, nblk, N, h->G32(boff));
+  k::partials_reduce_kernel<<<(N + 31) / 32, 256, 0, h->stream>>>(h->cs_part, nblk, N, N, h->G32(boff), nullptr,
+                                                                   nullptr);
   LAUNCH_CHECK(h);
   return GPT2_OK;
 }
