@@ -144,7 +144,33 @@ __device__ __forceinline__ void decode_tile(const Params& p, int tile, int& mb, 
   nb = t / p.num_m;
 }
 
+// 32-byte vector global accesses: one lane writes (or reads) a whole 32-byte
+// sector in one instruction.  Used when the row stride keeps every 32-column
+// chunk 32-byte aligned.
+__device__ __forceinline__ void st32(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                     uint32_t f, uint32_t g, uint32_t h) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d), "r"(e),
+               "r"(f), "r"(g), "r"(h)
+               : "memory");
+}
+__device__ __forceinline__ void ld32(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st_bf16x16(bf16* o, const float* v) {
+  st32(o, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]),
+       pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+}
+__device__ __forceinline__ void st_f32x8(float* o, const float* v) {
+  st32(o, __float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]),
+       __float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]), __float_as_uint(v[7]));
+}
+
 // ------------------------------------------------------------- epilogue
+// Fused math on the 32 consecutive columns [col0, col0+32) of one row.
+// FULL: all 32 columns lie inside N and every 32-column chunk is 32-byte
+// aligned (32-byte vector accesses); otherwise element-wise with masks.
 template <bool FULL>
 __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, int split, const uint32_t (&r)[32]) {
   float v[32];
@@ -160,22 +186,19 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
     case EPI_BF16: {
       bf16* o = reinterpret_cast<bf16*>(p.out) + base;
       if (FULL) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 w = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
-                               pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
-          *reinterpret_cast<uint4*>(o + i) = w;
-        }
+        st_bf16x16(o, v);
+        st_bf16x16(o + 16, v + 16);
       } else {
         for (int i = 0; i < 32; ++i)
           if (col0 + i < p.N) o[i] = f2bf(v[i]);
       }
     } break;
-    case EPI_F32: {
-      float* o = reinterpret_cast<float*>(p.out) + base;
+    case EPI_F32:
+    case EPI_PARTIAL_F32: {
+      float* o = (p.epi == EPI_F32 ? reinterpret_cast<float*>(p.out) : p.partial + (long)split * p.M * p.ldc) + base;
       if (FULL) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        for (int i = 0; i < 32; i += 8) st_f32x8(o + i, v + i);
       } else {
         for (int i = 0; i < 32; ++i)
           if (col0 + i < p.N) o[i] = v[i];
@@ -186,10 +209,14 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
       const float* rs = (p.epi == EPI_RESID_F32 ? p.resid : reinterpret_cast<const float*>(p.out)) + base;
       float* o = reinterpret_cast<float*>(p.out) + base;
       if (FULL) {
+        uint32_t x[4][8];
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float4 x = *reinterpret_cast<const float4*>(rs + i);
-          *reinterpret_cast<float4*>(o + i) = make_float4(x.x + v[i], x.y + v[i + 1], x.z + v[i + 2], x.w + v[i + 3]);
+        for (int i = 0; i < 4; ++i) ld32(rs + 8 * i, x[i]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[8 * i + e] += __uint_as_float(x[i][e]);
+          st_f32x8(o + 8 * i, v + 8 * i);
         }
       } else {
         for (int i = 0; i < 32; ++i)
@@ -199,26 +226,22 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
     case EPI_GELU: {
       bf16* o = reinterpret_cast<bf16*>(p.out) + base;
       bf16* o2 = p.out2 + base;
+      float u[32], g[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        u[i] = bf2f(f2bf(v[i]));  // the stored pre-activation, as rounded
+        g[i] = gelu_tanh<true>(u[i]);
+      }
       if (FULL) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          float u[8], g[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            u[j] = bf2f(f2bf(v[i + j]));  // the stored pre-activation, as rounded
-            g[j] = gelu_tanh<true>(u[j]);
-          }
-          *reinterpret_cast<uint4*>(o + i) = make_uint4(pack_bf16x2(u[0], u[1]), pack_bf16x2(u[2], u[3]),
-                                                        pack_bf16x2(u[4], u[5]), pack_bf16x2(u[6], u[7]));
-          *reinterpret_cast<uint4*>(o2 + i) = make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]),
-                                                         pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
-        }
+        st_bf16x16(o, u);
+        st_bf16x16(o + 16, u + 16);
+        st_bf16x16(o2, g);
+        st_bf16x16(o2 + 16, g + 16);
       } else {
         for (int i = 0; i < 32; ++i)
           if (col0 + i < p.N) {
-            float u = bf2f(f2bf(v[i]));
-            o[i] = f2bf(u);
-            o2[i] = f2bf(gelu_tanh<true>(u));
+            o[i] = f2bf(u[i]);
+            o2[i] = f2bf(g[i]);
           }
       }
     } break;
@@ -226,33 +249,22 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
       bf16* o = reinterpret_cast<bf16*>(p.out) + base;
       const bf16* ua = p.aux + base;
       if (FULL) {
+        uint32_t uw[2][8];
+        ld32(ua, uw[0]);
+        ld32(ua + 16, uw[1]);
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 uu = *reinterpret_cast<const uint4*>(ua + i);
-          uint32_t uw[4] = {uu.x, uu.y, uu.z, uu.w};
-          float d[8];
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float2 f = unpack_bf16x2(uw[j]);
-            d[2 * j] = v[i + 2 * j] * gelu_tanh_grad<true>(f.x);
-            d[2 * j + 1] = v[i + 2 * j + 1] * gelu_tanh_grad<true>(f.y);
+          for (int e = 0; e < 8; ++e) {
+            const float2 f = unpack_bf16x2(uw[h][e]);
+            v[16 * h + 2 * e] *= gelu_tanh_grad<true>(f.x);
+            v[16 * h + 2 * e + 1] *= gelu_tanh_grad<true>(f.y);
           }
-          *reinterpret_cast<uint4*>(o + i) = make_uint4(pack_bf16x2(d[0], d[1]), pack_bf16x2(d[2], d[3]),
-                                                        pack_bf16x2(d[4], d[5]), pack_bf16x2(d[6], d[7]));
-        }
+        st_bf16x16(o, v);
+        st_bf16x16(o + 16, v + 16);
       } else {
         for (int i = 0; i < 32; ++i)
           if (col0 + i < p.N) o[i] = f2bf(v[i] * gelu_tanh_grad<true>(bf2f(ua[i])));
-      }
-    } break;
-    case EPI_PARTIAL_F32: {
-      float* o = p.partial + (long)split * p.M * p.ldc + base;
-      if (FULL) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-      } else {
-        for (int i = 0; i < 32; ++i)
-          if (col0 + i < p.N) o[i] = v[i];
       }
     } break;
     default:
@@ -415,7 +427,7 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_ld();
         const int col0 = nb * BN + j * 32;
         if (row < p.M && col0 < p.N) {
-          if (col0 + 32 <= p.N)
+          if (col0 + 32 <= p.N && p.vec32)
             epi_store<true>(p, row, col0, split, r);
           else
             epi_store<false>(p, row, col0, split, r);
@@ -566,6 +578,18 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
   p.out2 = g.out2;
   p.aux = g.aux;
   p.ldc = g.ldc;
+  {
+    // 32-byte vector epilogue: every 32-column chunk of every row (and of the
+    // residual / aux / split-K partial buffers) must start on 32 bytes
+    const size_t es = (g.epi == EPI_BF16 || g.epi == EPI_GELU || g.epi == EPI_DGELU) ? 2 : 4;
+    auto al32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31) == 0; };
+    bool ok = (g.ldc * (long)es) % 32 == 0 && al32(g.out);
+    if (g.epi == EPI_RESID_F32) ok = ok && al32(g.resid);
+    if (g.epi == EPI_GELU) ok = ok && al32(g.out2);
+    if (g.epi == EPI_DGELU) ok = ok && al32(g.aux);
+    if (g.workspace) ok = ok && al32(g.workspace) && (g.ldc * 4L) % 32 == 0;
+    p.vec32 = ok ? 1 : 0;
+  }
   int splits = 1;
   if (g.epi == EPI_ACCUM_F32 && g.workspace != nullptr) {
     splits = choose_splits(p.num_m * p.num_n, p.kb_total);

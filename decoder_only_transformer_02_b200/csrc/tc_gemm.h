@@ -53,6 +53,7 @@ struct Params {
   const __nv_bfloat16* aux;
   long ldc;
   float* partial;
+  int vec32;  // 1: every 32-column chunk is 32-byte aligned (vector epilogue)
 };
 
 // Returns 0 on success, -1 bad arguments, -2 tensor-map encode failure, -3 launch failure.

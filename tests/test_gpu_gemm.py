@@ -46,7 +46,7 @@ def test_gemm_fp32_out_all_layouts(M, N, K, a_mn, b_mn):
     assert rel_max_err(from_dev(out), ref) < 1e-5
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 384, 200), (1000, 2304, 768)])
+@pytest.mark.parametrize("M,N,K", [(300, 384, 200), (1000, 2304, 768), (200, 136, 64)])
 def test_gemm_epilogues(M, N, K):
     from oracle import gpt2_oracle as O
     G = _lib()
