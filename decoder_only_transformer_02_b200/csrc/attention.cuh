@@ -13,11 +13,11 @@
 //   ds_ij = p_ij (dp_ij - D_i)      dq_i = sum_j ds_ij k_j / sqrt(d)
 //   dk_j = sum_i ds_ij q_i / sqrt(d)
 //
-// bf16 path (d = 64): flash-style tiling with the online softmax held in
-// registers, bf16 tensor-core MMAs (m16n8k16) with fp32 accumulation; S and P
-// never leave the chip.  The backward is two deterministic kernels (no atomics):
-// one owns a key block and produces dk, dv; the other owns a query block and
-// produces dq.
+// bf16 backward (d = 64): flash-style tiling, bf16 tensor-core MMAs (m16n8k16)
+// with fp32 accumulation; S and P never leave the chip.  Two deterministic
+// kernels (no atomics): one owns a key block and produces dk, dv; the other owns
+// a query block and produces dq.  (The bf16 forward is the tcgen05 kernel in
+// attention_tc.cuh.)
 // fp32 path: plain per-row kernels (fp32 parity mode, small shapes).
 #pragma once
 #include "common.cuh"
@@ -142,105 +142,6 @@ __device__ __forceinline__ void c_to_a(const float (&c)[8][4], uint32_t (&a)[4][
     a[kk][1] = pack_bf16x2(c[2 * kk][2], c[2 * kk][3]);
     a[kk][2] = pack_bf16x2(c[2 * kk + 1][0], c[2 * kk + 1][1]);
     a[kk][3] = pack_bf16x2(c[2 * kk + 1][2], c[2 * kk + 1][3]);
-  }
-}
-
-// ------------------------------------------------------------ forward
-__global__ void __launch_bounds__(128) flash_fwd_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ out,
-                                                        float* __restrict__ lse, int T, int H, float sl2) {
-  __shared__ __align__(128) uint8_t sQ[64 * 128];
-  __shared__ __align__(128) uint8_t sK[2][64 * 128];
-  __shared__ __align__(128) uint8_t sV[2][64 * 128];
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest (diagonal-heavy) blocks first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
-  const int C = H * HD;
-  const long ld = 3L * C;
-  const bf16* Qg = qkv + (long)b * T * ld + h * HD;
-  const bf16* Kg = Qg + C;
-  const bf16* Vg = Qg + 2 * C;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t4 = lane & 3;
-
-  load_tile(sQ, Qg, ld, qb * BQ, T);
-  load_tile(sK[0], Kg, ld, 0, T);
-  load_tile(sV[0], Vg, ld, 0, T);
-  cp_commit();
-
-  uint32_t qf[4][4];
-  float o[8][4] = {};
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  const int q_row0 = qb * BQ + warp * 16 + g;  // this thread's rows: q_row0, q_row0 + 8
-  const int nkv = qb + 1;
-
-  for (int j = 0; j < nkv; ++j) {
-    cp_wait<0>();
-    __syncthreads();
-    if (j + 1 < nkv) {
-      load_tile(sK[(j + 1) & 1], Kg, ld, (j + 1) * BKV, T);
-      load_tile(sV[(j + 1) & 1], Vg, ld, (j + 1) * BKV, T);
-    }
-    cp_commit();
-    if (j == 0) load_a_frags(sQ, warp * 16, qf);
-    float s[8][4] = {};
-    mma_a_bt(s, qf, sK[j & 1]);
-    // scale to log2 units and mask
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = s[nt][e] * sl2;
-        if (j == qb) {
-          const int key = j * BKV + nt * 8 + 2 * t4 + (e & 1);
-          const int qr = q_row0 + ((e >> 1) << 3);
-          if (key > qr) v = -INFINITY;
-        }
-        s[nt][e] = v;
-      }
-    // online softmax (rows g and g+8)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * hr], s[nt][2 * hr + 1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_r[hr], mx);
-      const float alpha = ex2(m_r[hr] - m_new);
-      float rs = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        s[nt][2 * hr] = ex2(s[nt][2 * hr] - m_new);
-        s[nt][2 * hr + 1] = ex2(s[nt][2 * hr + 1] - m_new);
-        rs += s[nt][2 * hr] + s[nt][2 * hr + 1];
-      }
-      l_r[hr] = l_r[hr] * alpha + rs;
-      m_r[hr] = m_new;
-#pragma unroll
-      for (int dt = 0; dt < 8; ++dt) {
-        o[dt][2 * hr] *= alpha;
-        o[dt][2 * hr + 1] *= alpha;
-      }
-    }
-    uint32_t pf[4][4];
-    c_to_a(s, pf);
-    mma_a_b(o, pf, sV[j & 1]);
-  }
-  // finalize: full row sums across the 4 threads of a row
-#pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    float l = l_r[hr];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const int qr = q_row0 + hr * 8;
-    const float inv = 1.f / l;
-    if (qr < T) {
-      bf16* orow = out + ((long)b * T + qr) * C + h * HD;
-#pragma unroll
-      for (int dt = 0; dt < 8; ++dt)
-        *reinterpret_cast<uint32_t*>(orow + dt * 8 + 2 * t4) =
-            pack_bf16x2(o[dt][2 * hr] * inv, o[dt][2 * hr + 1] * inv);
-      if (t4 == 0) lse[((long)b * H + h) * T + qr] = (m_r[hr] + __log2f(l)) * LN2;
-    }
   }
 }
 
@@ -439,14 +340,6 @@ __global__ void __launch_bounds__(128) flash_bwd_dq_kernel(const bf16* __restric
             pack_bf16x2(dq[dt][2 * hr] * scale, dq[dt][2 * hr + 1] * scale);
     }
   }
-}
-
-static inline cudaError_t flash_forward(const bf16* qkv, bf16* out, float* lse, int B, int T, int H,
-                                        cudaStream_t st) {
-  const float sl2 = LOG2E / sqrtf((float)HD);
-  dim3 grid((T + BQ - 1) / BQ, B * H);
-  flash_fwd_kernel<<<grid, 128, 0, st>>>(qkv, out, lse, T, H, sl2);
-  return cudaGetLastError();
 }
 
 // Dv: caller-provided fp32 scratch of B*H*T elements

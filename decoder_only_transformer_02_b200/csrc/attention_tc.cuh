@@ -1,0 +1,331 @@
+// Causal attention forward on the 5th-generation tensor cores (tcgen05).
+//
+// Same contract as attn::flash_forward (bf16 qkv [B, T, 3C], head dim 64,
+// output o [B, T, C] bf16 and lse [B, H, T] fp32).  One CTA owns 128 queries
+// of one (batch, head) and walks the key blocks 0..qb of 128 keys:
+//   S_j  = Q K_j^T        tcgen05.mma, M=128 x N=128 x K=64, fp32 in TMEM
+//   P_j  = exp(S_j/sqrt(d) - m_j)  (online softmax, one thread per query row,
+//          read from TMEM; bf16 P written to shared memory in the 128-byte
+//          swizzled K-major layout the MMA reads)
+//   PV_j = P_j V_j        tcgen05.mma, M=128 x N=64 x K=128, fp32 in TMEM
+//   O    = alpha_j (O + PV_{j-1}) in registers, O/l at the end.
+// Warp 0 loads Q once and K_j, V_j through a 3-stage TMA ring; warp 1 issues
+// the MMAs (S_{j+1} is computed while the softmax warps work on S_j); warps
+// 2..5 do the softmax (warp w reads TMEM lanes 32*(w%4)..+31).  S and PV are
+// double-buffered in TMEM.  All waits are bounded.
+#pragma once
+#include "common.cuh"
+
+namespace tcfa {
+
+using namespace tcg;
+
+constexpr int BQ = 128;       // queries per CTA
+constexpr int BKV = 128;      // keys per block
+constexpr int HD = 64;        // head dim
+constexpr int KV_STAGES = 3;
+constexpr int TILE = 128 * 64 * 2;          // one 128 x 64 bf16 tile (16 KB)
+constexpr int Q_OFF = 0;
+constexpr int KV_OFF = TILE;                // stage s: K at +2s*TILE, V at +(2s+1)*TILE
+constexpr int P_OFF = KV_OFF + 2 * KV_STAGES * TILE;  // two P buffers of 2 tiles each
+constexpr int BAR_OFF = P_OFF + 4 * TILE;
+constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
+constexpr uint32_t TMEM_COLS = 512;         // S0 0, S1 128, PV0 256, PV1 320
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// byte offset of element (r, c) in a 128-row, 64-column bf16 K-major tile with
+// the 128-byte swizzle (16-byte chunk c/8 of row r stored at chunk (c/8)^(r%8))
+__device__ __forceinline__ uint32_t sw128(int r, int chunk) {
+  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(192, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse, int T,
+               int H, float sl2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* q_full = bars;                 // 1
+  uint64_t* kv_full = bars + 1;            // KV_STAGES
+  uint64_t* kv_empty = kv_full + KV_STAGES;
+  uint64_t* s_full = kv_empty + KV_STAGES;  // 2
+  uint64_t* s_free = s_full + 2;            // 2 (count 4)
+  uint64_t* p_full = s_free + 2;            // 2 (count 4)
+  uint64_t* pv_full = p_full + 2;           // 2
+  uint64_t* pv_free = pv_full + 2;          // 2 (count 4)
+  uint64_t* drain = pv_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = gridDim.x - 1 - blockIdx.x;  // longest blocks first
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int nkv = qb + 1;
+  const int row0 = b * T;  // first row of this batch in the [B*T, 3C] view
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_full[i], 1);
+      mbar_init(&pv_free[i], 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      mbar_expect_tx(q_full, TILE);
+      tma_load_2d(smem_u32(smem + Q_OFF), &tm_qkv, h * HD, row0 + qb * BQ, q_full);
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j, ++issued) {
+        const int s = j % KV_STAGES;
+        if (!mbar_wait(&kv_empty[s], ((j / KV_STAGES) & 1u) ^ 1u)) {
+          set_device_err(DERR_WAIT_TIMEOUT);
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(&kv_full[s], 2 * TILE);
+        const uint32_t kd = smem_u32(smem + KV_OFF + 2 * s * TILE);
+        tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + j * BKV, &kv_full[s]);
+        tma_load_2d(kd + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BKV, &kv_full[s]);
+      }
+      (void)ok;
+      // drain: every issued K/V load has been consumed by its PV MMA
+      for (int s = 0; s < KV_STAGES; ++s) {
+        if ((uint32_t)s < issued) {
+          const uint32_t last = issued - 1 - ((issued - 1 - s) % KV_STAGES);
+          if (!mbar_wait(&kv_empty[s], (last / KV_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        }
+      }
+      if (!mbar_wait(q_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      // S: A = Q (K-major), B = K_j (K-major), M=128, N=128
+      const uint32_t id_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BKV >> 3) << 17) |
+                            ((uint32_t)(BQ >> 4) << 24);
+      // PV: A = P_j (K-major over keys), B = V_j (MN-major: d contiguous), M=128, N=64
+      const uint32_t id_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(HD >> 3) << 17) |
+                             ((uint32_t)(BQ >> 4) << 24);
+      bool ok = mbar_wait(q_full, 0);
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_fence_after();
+      const uint32_t qa = smem_u32(smem + Q_OFF);
+      auto do_pv = [&](int i) -> bool {
+        const int pb = i & 1;
+        if (!mbar_wait(&p_full[pb], (i >> 1) & 1u)) return false;
+        if (i >= 2 && !mbar_wait(&pv_free[pb], ((i - 2) >> 1) & 1u)) return false;
+        tc_fence_after();
+        const int s = i % KV_STAGES;
+        const uint32_t pa = smem_u32(smem + P_OFF + pb * 2 * TILE);
+        const uint32_t va = smem_u32(smem + KV_OFF + (2 * s + 1) * TILE);
+        const uint32_t d = tmem + 256 + pb * HD;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint64_t ad = make_sdesc(pa + (kk >> 2) * TILE + (kk & 3) * 32, 0);
+          const uint64_t bd = make_sdesc(va + kk * 2048, 1);
+          tc_mma(d, ad, bd, id_pv, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&pv_full[pb]);
+        tc_commit(&kv_empty[s]);
+        return true;
+      };
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % KV_STAGES, sb = j & 1;
+        if (!mbar_wait(&kv_full[s], (j / KV_STAGES) & 1u)) {
+          ok = false;
+          break;
+        }
+        if (j >= 2 && !mbar_wait(&s_free[sb], ((j - 2) >> 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ka = smem_u32(smem + KV_OFF + 2 * s * TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint64_t ad = make_sdesc(qa + kk * 32, 0);
+          const uint64_t bd = make_sdesc(ka + kk * 32, 0);
+          tc_mma(tmem + sb * BKV, ad, bd, id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[sb]);
+        if (j >= 1 && !do_pv(j - 1)) ok = false;
+      }
+      if (ok && !do_pv(nkv - 1)) ok = false;
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_commit(drain);
+      if (!mbar_wait(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------- softmax warps
+    const int qw = warp & 3;                // TMEM lane quarter
+    const int r = qw * 32 + lane;           // query row within the block
+    const int q = qb * BQ + r;              // query position in the sequence
+    const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+    float o[HD];
+#pragma unroll
+    for (int i = 0; i < HD; ++i) o[i] = 0.f;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait(&s_full[sb], (j >> 1) & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = (j == qb);
+      // the whole 128-key row of S in registers (one TMEM wait), buffer released
+      uint32_t v[BKV];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tl + sb * BKV + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+      // row maximum of the raw scores (masked keys excluded), 8 independent
+      // chains; the scale 1/sqrt(d)*log2(e) > 0 is applied to the maximum
+      if (diag) {
+#pragma unroll
+        for (int e = 0; e < BKV; ++e)
+          if (j * BKV + e > q) v[e] = __float_as_uint(-INFINITY);
+      }
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(v[i]);
+#pragma unroll
+      for (int e = 8; e < BKV; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_new = fmaxf(m, mx * sl2);
+      const float alpha = ex2f(m - m_new);
+      // probabilities p = 2^(s*sl2 - m_new) (one FFMA + ex2), row sum in 8
+      // chains, bf16 P into shared memory
+      float rs8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
+      uint8_t* pbuf = smem + P_OFF + sb * 2 * TILE;
+#pragma unroll
+      for (int k = 0; k < BKV / 8; ++k) {
+        float pv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pv[e] = ex2f(fmaf(__uint_as_float(v[8 * k + e]), sl2, -m_new));
+          rs8[e] += pv[e];
+        }
+        const uint4 w = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
+                                   pack_bf16x2(pv[6], pv[7]));
+        // keys 8k..8k+7: tile half k/8, 16-byte chunk k%8
+        *reinterpret_cast<uint4*>(pbuf + (k >> 3) * TILE + sw128(r, k & 7)) = w;
+      }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+      l = l * alpha + rs;
+      m = m_new;
+      if (j >= 1) {
+        const int pb = (j - 1) & 1;
+        if (!mbar_wait(&pv_full[pb], ((j - 1) >> 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t a0[32], a1[32];
+        tmem_ld32(tl + 256 + pb * HD, a0);
+        tmem_ld32(tl + 256 + pb * HD + 32, a1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pv_free[pb]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          o[i] = (o[i] + __uint_as_float(a0[i])) * alpha;
+          o[32 + i] = (o[32 + i] + __uint_as_float(a1[i])) * alpha;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < HD; ++i) o[i] *= alpha;
+      }
+    }
+    if (ok) {
+      const int pb = (nkv - 1) & 1;
+      if (mbar_wait(&pv_full[pb], ((nkv - 1) >> 1) & 1u)) {
+        tc_fence_after();
+        uint32_t a0[32], a1[32];
+        tmem_ld32(tl + 256 + pb * HD, a0);
+        tmem_ld32(tl + 256 + pb * HD + 32, a1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          o[i] += __uint_as_float(a0[i]);
+          o[32 + i] += __uint_as_float(a1[i]);
+        }
+        if (q < T) {
+          const float inv = 1.f / l;
+          bf16* orow = out + ((long)b * T + q) * C + h * HD;
+#pragma unroll
+          for (int i = 0; i < HD; i += 8)
+            *reinterpret_cast<uint4*>(orow + i) =
+                make_uint4(pack_bf16x2(o[i] * inv, o[i + 1] * inv), pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv),
+                           pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv), pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv));
+          lse[((long)b * H + h) * T + q] = (m + __log2f(l)) * 0.6931471805599453f;
+        }
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+static inline cudaError_t forward(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap tm;
+  const int C = H * HD;
+  if (make_tmap(&tm, qkv, 3L * C, (long)B * T, 3L * C, 64, 128) != 0) return cudaErrorInvalidValue;
+  const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
+  dim3 grid((T + BQ - 1) / BQ, B * H);
+  fwd_kernel<<<grid, 192, SMEM_BYTES, st>>>(tm, out, lse, T, H, sl2);
+  return cudaGetLastError();
+}
+
+}  // namespace tcfa

@@ -2,6 +2,7 @@
 // kernels, the GEMM and the runtime are all included here so that they share
 // one device error word.
 #include "tc_gemm.cu"
+#include "attention_tc.cuh"
 #include "model_pass.cuh"
 
 #include <mutex>
@@ -283,7 +284,7 @@ int gpt2_attention_forward(const void* qkv, void* out, float* lse, int B, int T,
   if (!qkv || !out || !lse || B < 1 || T < 1 || H < 1) return GPT2_EINVAL;
   if (!aligned16(qkv) || !aligned16(out)) return GPT2_EINVAL;
   if ((long)B * H > 65535L * 1024) return GPT2_EINVAL;
-  return attn::flash_forward((const bf16*)qkv, (bf16*)out, lse, B, T, H, (cudaStream_t)stream) == cudaSuccess
+  return tcfa::forward((const bf16*)qkv, (bf16*)out, lse, B, T, H, (cudaStream_t)stream) == cudaSuccess
              ? GPT2_OK
              : GPT2_ECUDA;
 }

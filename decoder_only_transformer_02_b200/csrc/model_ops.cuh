@@ -228,7 +228,7 @@ static int op_attn_fwd(gpt2* h, int l) {
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;
   (void)M;
   if (h->prec == GPT2_BF16) {
-    if (attn::flash_forward((const bf16*)qkv, (bf16*)att, lse, h->B, h->T, h->H, h->stream) != cudaSuccess)
+    if (tcfa::forward((const bf16*)qkv, (bf16*)att, lse, h->B, h->T, h->H, h->stream) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention forward launch");
     h->launches++;
   } else {

@@ -178,9 +178,20 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
   const long base = (long)row * p.ldc + col0;
   if (p.bias != nullptr && p.epi != EPI_DGELU && p.epi != EPI_ACCUM_F32 && p.epi != EPI_PARTIAL_F32) {
+    if (FULL) {
+      const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (FULL || col0 + i < p.N) v[i] += __ldg(p.bias + col0 + i);
+      for (int i = 0; i < 8; ++i) {
+        const float4 b = __ldg(b4 + i);
+        v[4 * i] += b.x;
+        v[4 * i + 1] += b.y;
+        v[4 * i + 2] += b.z;
+        v[4 * i + 3] += b.w;
+      }
+    } else {
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < p.N) v[i] += __ldg(p.bias + col0 + i);
+    }
   }
   switch (p.epi) {
     case EPI_BF16: {
@@ -420,22 +431,30 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int row = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      // 64 accumulator columns per TMEM wait; the buffer is handed back to the
+      // MMA warp as soon as its last columns are in registers
 #pragma unroll 1
-      for (int j = 0; j < BN / 32; ++j) {
-        uint32_t r[32];
-        tmem_ld32(tbase + j * 32, r);
+      for (int j = 0; j < BN / 64; ++j) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tbase + j * 64, r0);
+        tmem_ld32(tbase + j * 64 + 32, r1);
         tmem_wait_ld();
-        const int col0 = nb * BN + j * 32;
-        if (row < p.M && col0 < p.N) {
-          if (col0 + 32 <= p.N && p.vec32)
-            epi_store<true>(p, row, col0, split, r);
-          else
-            epi_store<false>(p, row, col0, split, r);
+        if (j == BN / 64 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int col0 = nb * BN + j * 64 + h * 32;
+          if (row < p.M && col0 < p.N) {
+            if (col0 + 32 <= p.N && p.vec32)
+              epi_store<true>(p, row, col0, split, h ? r1 : r0);
+            else
+              epi_store<false>(p, row, col0, split, h ? r1 : r0);
+          }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
     }
   }
   __syncthreads();
