@@ -1,7 +1,7 @@
 // Causal attention forward on the 5th-generation tensor cores (tcgen05).
 //
-// Same contract as attn::flash_forward (bf16 qkv [B, T, 3C], head dim 64,
-// output o [B, T, C] bf16 and lse [B, H, T] fp32).  One CTA owns 128 queries
+// bf16 qkv [B, T, 3C] (q, k, v column blocks, head h in columns h*64..),
+// head dim 64; output o [B, T, C] bf16 and lse [B, H, T] fp32.  One CTA owns 128 queries
 // of one (batch, head) and walks the key blocks 0..qb of 128 keys:
 //   S_j  = Q K_j^T        tcgen05.mma, M=128 x N=128 x K=64, fp32 in TMEM
 //   P_j  = exp(S_j/sqrt(d) - m_j)  (online softmax, one thread per query row,

@@ -1,0 +1,508 @@
+// Causal attention backward on tcgen05 (bf16 operands, fp32 TMEM accumulators).
+//
+// With P = exp(S/sqrt(d) - lse), D_q = sum_d dO_q . O_q (precomputed):
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dK = dS^T Q / sqrt(d),
+//   dQ = dS K / sqrt(d).
+// Two deterministic kernels (no atomics), in the structure of the forward:
+//  dkdv_kernel: one CTA owns 128 keys and walks the query blocks i >= kb:
+//     S^T = K Q_i^T and dP^T = V dO_i^T (M=128 keys, N=128 queries, K=64) into
+//     TMEM; four compute warps (one key row per thread) form bf16 P^T and dS^T
+//     in shared memory (128-byte swizzled, K-major over queries); then
+//     dV += P^T dO_i and dK += dS^T Q_i (M=128, N=64, K=128) accumulate in TMEM.
+//  dq_kernel: one CTA owns 128 queries and walks the key blocks j <= qb:
+//     S = Q K_j^T, dP = dO V_j^T, dS = P * (dP - D) (one query row per thread),
+//     dQ += dS K_j.
+// Q_i / dO_i (resp. K_j / V_j) stream through a 2-stage TMA ring; the same
+// swizzled tile serves as a K-major operand (contraction over d) and as an
+// MN-major one (contraction over its rows).
+#pragma once
+#include "attention.cuh"
+#include "attention_tc.cuh"
+
+namespace tcfa {
+
+constexpr int B_STAGES = 2;
+
+// ------------------------------------------------------------ dK, dV
+constexpr int DKV_K_OFF = 0;
+constexpr int DKV_V_OFF = TILE;
+constexpr int DKV_RING_OFF = 2 * TILE;                     // stage s: Q at +2s*TILE, dO at +(2s+1)*TILE
+constexpr int DKV_P_OFF = DKV_RING_OFF + 2 * B_STAGES * TILE;  // P^T: 2 tiles
+constexpr int DKV_DS_OFF = DKV_P_OFF + 2 * TILE;            // dS^T: 2 tiles
+constexpr int DKV_LD_OFF = DKV_DS_OFF + 2 * TILE;           // stage s: lse*log2(e)[128], D[128]
+constexpr int DKV_BAR_OFF = DKV_LD_OFF + B_STAGES * 1024;
+constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                const float* __restrict__ lse, const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H,
+                float scale, float sl2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
+  uint64_t* kv_full = bars;                // K and V tiles
+  uint64_t* qd_full = bars + 1;            // B_STAGES
+  uint64_t* qd_empty = qd_full + B_STAGES;
+  uint64_t* s_full = qd_empty + B_STAGES;  // S^T and dP^T ready
+  uint64_t* s_free = s_full + 1;           // count 4
+  uint64_t* p_full = s_free + 1;           // count 4
+  uint64_t* acc_done = p_full + 1;
+  uint64_t* ld_full = acc_done + 1;        // B_STAGES: lse / D of the stage's queries
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ld_full + B_STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb = blockIdx.x;  // key block; small kb = most query blocks, launched first
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int nqb = (T + BQ - 1) / BQ;
+  const int row0 = b * T;
+  const int nblk = nqb - kb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < B_STAGES; ++s) {
+      mbar_init(&qd_full[s], 1);
+      mbar_init(&qd_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(acc_done, 1);
+    for (int s = 0; s < B_STAGES; ++s) mbar_init(&ld_full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // S^T at 0, dP^T at 128, dV at 256, dK at 320
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    // lane 0 drives the TMA ring; the whole warp stages each query block's
+    // lse (log2 units; +inf past T) and D (0 past T) next to its Q / dO tiles
+    if (lane == 0) {
+      mbar_expect_tx(kv_full, 2 * TILE);
+      tma_load_2d(smem_u32(smem + DKV_K_OFF), &tm_qkv, C + h * HD, row0 + kb * BKV, kv_full);
+      tma_load_2d(smem_u32(smem + DKV_V_OFF), &tm_qkv, 2 * C + h * HD, row0 + kb * BKV, kv_full);
+    }
+    const float* lrow = lse + ((long)b * H + h) * T;
+    const float* drow = Dv + ((long)b * H + h) * T;
+    uint32_t issued = 0;
+    for (int n = 0; n < nblk; ++n, ++issued) {
+      const int i = kb + n, s = n % B_STAGES;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&qd_empty[s], ((n / B_STAGES) & 1u) ^ 1u) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        if (lane == 0) set_device_err(DERR_WAIT_TIMEOUT);
+        break;
+      }
+      float* ld = reinterpret_cast<float*>(smem + DKV_LD_OFF + s * 1024);
+      for (int c = lane; c < BQ; c += 32) {
+        const int q = i * BQ + c;
+        ld[c] = q < T ? lrow[q] * 1.4426950408889634f : INFINITY;
+        ld[BQ + c] = q < T ? drow[q] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&ld_full[s]);
+        mbar_expect_tx(&qd_full[s], 2 * TILE);
+        const uint32_t dst = smem_u32(smem + DKV_RING_OFF + 2 * s * TILE);
+        tma_load_2d(dst, &tm_qkv, h * HD, row0 + i * BQ, &qd_full[s]);
+        tma_load_2d(dst + TILE, &tm_do, h * HD, row0 + i * BQ, &qd_full[s]);
+      }
+    }
+    if (lane == 0) {
+      for (int s = 0; s < B_STAGES; ++s) {
+        if ((uint32_t)s < issued) {
+          const uint32_t last = issued - 1 - ((issued - 1 - s) % B_STAGES);
+          if (!mbar_wait(&qd_empty[s], (last / B_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        }
+      }
+      if (!mbar_wait(kv_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      const uint32_t id_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BQ >> 3) << 17) |
+                            ((uint32_t)(BKV >> 4) << 24);
+      const uint32_t id_acc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(HD >> 3) << 17) |
+                              ((uint32_t)(BKV >> 4) << 24);
+      bool ok = mbar_wait(kv_full, 0);
+      const uint32_t ka = smem_u32(smem + DKV_K_OFF), va = smem_u32(smem + DKV_V_OFF);
+      const uint32_t pa = smem_u32(smem + DKV_P_OFF), dsa = smem_u32(smem + DKV_DS_OFF);
+      for (int n = 0; ok && n < nblk; ++n) {
+        const int s = n % B_STAGES;
+        if (!mbar_wait(&qd_full[s], (n / B_STAGES) & 1u)) {
+          ok = false;
+          break;
+        }
+        if (n >= 1 && !mbar_wait(s_free, (n - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t qa = smem_u32(smem + DKV_RING_OFF + 2 * s * TILE);
+        const uint32_t doa = qa + TILE;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          tc_mma(tmem, make_sdesc(ka + kk * 32, 0), make_sdesc(qa + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + 128, make_sdesc(va + kk * 32, 0), make_sdesc(doa + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        if (!mbar_wait(p_full, n & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+          tc_mma(tmem + 256, make_sdesc(pa + aoff, 0), make_sdesc(doa + kk * 2048, 1), id_acc, acc);
+          tc_mma(tmem + 320, make_sdesc(dsa + aoff, 0), make_sdesc(qa + kk * 2048, 1), id_acc, acc);
+        }
+        tc_commit(&qd_empty[s]);
+      }
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_commit(acc_done);
+      if (!mbar_wait(acc_done, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------- compute warps
+    const int qw = warp & 3;
+    const int kr = qw * 32 + lane;            // key row within the block
+    const int key = kb * BKV + kr;            // key position
+    const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+    bool ok = true;
+    for (int n = 0; n < nblk; ++n) {
+      const int i = kb + n, s = n % B_STAGES;
+      if (!mbar_wait(&ld_full[s], (n / B_STAGES) & 1u) || !mbar_wait(s_full, n & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = (i == kb);
+      const float* ldl = reinterpret_cast<const float*>(smem + DKV_LD_OFF + s * 1024);
+      uint8_t* pt = smem + DKV_P_OFF;
+      uint8_t* dst = smem + DKV_DS_OFF;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[64], dv[64];
+        tmem_ld32(tl + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tl + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tl + 128 + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+        tmem_ld32(tl + 128 + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c0 = hh * 64 + 8 * k;
+          const int q0 = i * BQ + c0;
+          const float4 la = *reinterpret_cast<const float4*>(ldl + c0);
+          const float4 lb = *reinterpret_cast<const float4*>(ldl + c0 + 4);
+          const float4 da = *reinterpret_cast<const float4*>(ldl + BQ + c0);
+          const float4 db = *reinterpret_cast<const float4*>(ldl + BQ + c0 + 4);
+          const float l8[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+          const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          float p[8], ds[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float pe = ex2f(fmaf(__uint_as_float(sv[8 * k + e]), sl2, -l8[e]));
+            if (diag && (q0 + e < key)) pe = 0.f;
+            p[e] = pe;
+            ds[e] = pe * (__uint_as_float(dv[8 * k + e]) - d8[e]);
+          }
+          *reinterpret_cast<uint4*>(pt + hh * TILE + sw128(kr, k)) =
+              make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                         pack_bf16x2(p[6], p[7]));
+          *reinterpret_cast<uint4*>(dst + hh * TILE + sw128(kr, k)) =
+              make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
+                         pack_bf16x2(ds[6], ds[7]));
+        }
+      }
+      tc_fence_before();
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(s_free);
+        mbar_arrive(p_full);
+      }
+    }
+    if (ok && mbar_wait(acc_done, 0)) {
+      tc_fence_after();
+      uint32_t a[64];
+      tmem_ld32(tl + 256, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+      tmem_ld32(tl + 288, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+      tmem_wait_ld();
+      if (key < T) {
+        bf16* vrow = dqkv + ((long)b * T + key) * (3L * C) + 2 * C + h * HD;
+#pragma unroll
+        for (int e = 0; e < HD; e += 8)
+          *reinterpret_cast<uint4*>(vrow + e) = make_uint4(
+              pack_bf16x2(__uint_as_float(a[e]), __uint_as_float(a[e + 1])),
+              pack_bf16x2(__uint_as_float(a[e + 2]), __uint_as_float(a[e + 3])),
+              pack_bf16x2(__uint_as_float(a[e + 4]), __uint_as_float(a[e + 5])),
+              pack_bf16x2(__uint_as_float(a[e + 6]), __uint_as_float(a[e + 7])));
+      }
+      tmem_ld32(tl + 320, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+      tmem_ld32(tl + 352, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+      tmem_wait_ld();
+      if (key < T) {
+        bf16* krow = dqkv + ((long)b * T + key) * (3L * C) + C + h * HD;
+#pragma unroll
+        for (int e = 0; e < HD; e += 8)
+          *reinterpret_cast<uint4*>(krow + e) = make_uint4(
+              pack_bf16x2(__uint_as_float(a[e]) * scale, __uint_as_float(a[e + 1]) * scale),
+              pack_bf16x2(__uint_as_float(a[e + 2]) * scale, __uint_as_float(a[e + 3]) * scale),
+              pack_bf16x2(__uint_as_float(a[e + 4]) * scale, __uint_as_float(a[e + 5]) * scale),
+              pack_bf16x2(__uint_as_float(a[e + 6]) * scale, __uint_as_float(a[e + 7]) * scale));
+      }
+    } else {
+      ok = false;
+    }
+    if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ----------------------------------------------------------------- dQ
+constexpr int DQ_Q_OFF = 0;
+constexpr int DQ_DO_OFF = TILE;
+constexpr int DQ_RING_OFF = 2 * TILE;                      // stage s: K at +2s*TILE, V at +(2s+1)*TILE
+constexpr int DQ_DS_OFF = DQ_RING_OFF + 2 * B_STAGES * TILE;  // dS: 2 tiles
+constexpr int DQ_BAR_OFF = DQ_DS_OFF + 2 * TILE;
+constexpr int DQ_SMEM = DQ_BAR_OFF + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+              const float* __restrict__ lse, const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H,
+              float scale, float sl2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
+  uint64_t* q_full = bars;                 // Q and dO tiles
+  uint64_t* kv_full = bars + 1;            // B_STAGES
+  uint64_t* kv_empty = kv_full + B_STAGES;
+  uint64_t* s_full = kv_empty + B_STAGES;
+  uint64_t* s_free = s_full + 1;           // count 4
+  uint64_t* p_full = s_free + 1;           // count 4
+  uint64_t* acc_done = p_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = gridDim.x - 1 - blockIdx.x;  // most key blocks first
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int row0 = b * T;
+  const int nblk = qb + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < B_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(acc_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // S at 0, dP at 128, dQ at 256
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      mbar_expect_tx(q_full, 2 * TILE);
+      tma_load_2d(smem_u32(smem + DQ_Q_OFF), &tm_qkv, h * HD, row0 + qb * BQ, q_full);
+      tma_load_2d(smem_u32(smem + DQ_DO_OFF), &tm_do, h * HD, row0 + qb * BQ, q_full);
+      uint32_t issued = 0;
+      for (int j = 0; j < nblk; ++j, ++issued) {
+        const int s = j % B_STAGES;
+        if (!mbar_wait(&kv_empty[s], ((j / B_STAGES) & 1u) ^ 1u)) {
+          set_device_err(DERR_WAIT_TIMEOUT);
+          break;
+        }
+        mbar_expect_tx(&kv_full[s], 2 * TILE);
+        const uint32_t dst = smem_u32(smem + DQ_RING_OFF + 2 * s * TILE);
+        tma_load_2d(dst, &tm_qkv, C + h * HD, row0 + j * BKV, &kv_full[s]);
+        tma_load_2d(dst + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BKV, &kv_full[s]);
+      }
+      for (int s = 0; s < B_STAGES; ++s) {
+        if ((uint32_t)s < issued) {
+          const uint32_t last = issued - 1 - ((issued - 1 - s) % B_STAGES);
+          if (!mbar_wait(&kv_empty[s], (last / B_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        }
+      }
+      if (!mbar_wait(q_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      const uint32_t id_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BKV >> 3) << 17) |
+                            ((uint32_t)(BQ >> 4) << 24);
+      const uint32_t id_acc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(HD >> 3) << 17) |
+                              ((uint32_t)(BQ >> 4) << 24);
+      bool ok = mbar_wait(q_full, 0);
+      const uint32_t qa = smem_u32(smem + DQ_Q_OFF), doa = smem_u32(smem + DQ_DO_OFF);
+      const uint32_t dsa = smem_u32(smem + DQ_DS_OFF);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int s = j % B_STAGES;
+        if (!mbar_wait(&kv_full[s], (j / B_STAGES) & 1u)) {
+          ok = false;
+          break;
+        }
+        if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ka = smem_u32(smem + DQ_RING_OFF + 2 * s * TILE);
+        const uint32_t va = ka + TILE;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          tc_mma(tmem, make_sdesc(qa + kk * 32, 0), make_sdesc(ka + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + 128, make_sdesc(doa + kk * 32, 0), make_sdesc(va + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        if (!mbar_wait(p_full, j & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+          tc_mma(tmem + 256, make_sdesc(dsa + aoff, 0), make_sdesc(ka + kk * 2048, 1), id_acc,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&kv_empty[s]);
+      }
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_commit(acc_done);
+      if (!mbar_wait(acc_done, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------- compute warps
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;  // query row within the block
+    const int q = qb * BQ + r;
+    const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+    const float l2 = q < T ? lse[((long)b * H + h) * T + q] * 1.4426950408889634f : INFINITY;
+    const float dq_ = q < T ? Dv[((long)b * H + h) * T + q] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      if (!mbar_wait(s_full, j & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = (j == qb);
+      uint8_t* dst = smem + DQ_DS_OFF;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[64], dv[64];
+        tmem_ld32(tl + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tl + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tl + 128 + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+        tmem_ld32(tl + 128 + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float ds[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int key = j * BKV + hh * 64 + 8 * k + e;
+            float pe = ex2f(fmaf(__uint_as_float(sv[8 * k + e]), sl2, -l2));
+            if (diag && key > q) pe = 0.f;
+            ds[e] = pe * (__uint_as_float(dv[8 * k + e]) - dq_);
+          }
+          *reinterpret_cast<uint4*>(dst + hh * TILE + sw128(r, k)) =
+              make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
+                         pack_bf16x2(ds[6], ds[7]));
+        }
+      }
+      tc_fence_before();
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(s_free);
+        mbar_arrive(p_full);
+      }
+    }
+    if (ok && mbar_wait(acc_done, 0)) {
+      tc_fence_after();
+      uint32_t a[64];
+      tmem_ld32(tl + 256, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+      tmem_ld32(tl + 288, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+      tmem_wait_ld();
+      if (q < T) {
+        bf16* qrow = dqkv + ((long)b * T + q) * (3L * C) + h * HD;
+#pragma unroll
+        for (int e = 0; e < HD; e += 8)
+          *reinterpret_cast<uint4*>(qrow + e) = make_uint4(
+              pack_bf16x2(__uint_as_float(a[e]) * scale, __uint_as_float(a[e + 1]) * scale),
+              pack_bf16x2(__uint_as_float(a[e + 2]) * scale, __uint_as_float(a[e + 3]) * scale),
+              pack_bf16x2(__uint_as_float(a[e + 4]) * scale, __uint_as_float(a[e + 5]) * scale),
+              pack_bf16x2(__uint_as_float(a[e + 6]) * scale, __uint_as_float(a[e + 7]) * scale));
+      }
+    } else {
+      ok = false;
+    }
+    if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// D = rowsum(dO * O) (attn::bwd_dot_kernel), then the two kernels above.
+// Dv: caller-provided fp32 scratch of B*H*T elements.
+static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, bf16* dqkv,
+                                   float* Dv, int B, int T, int H, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int C = H * HD;
+  CUtensorMap tq, td;
+  if (make_tmap(&tq, qkv, 3L * C, (long)B * T, 3L * C, 64, 128) != 0) return cudaErrorInvalidValue;
+  if (make_tmap(&td, dout, C, (long)B * T, C, 64, 128) != 0) return cudaErrorInvalidValue;
+  const long rows = (long)B * T * H;
+  int blocks = (int)((rows * 32 + 255) / 256);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  attn::bwd_dot_kernel<<<blocks, 256, 0, st>>>(out, dout, Dv, B, T, H);
+  const float scale = 1.f / sqrtf((float)HD);
+  const float sl2 = 1.4426950408889634f * scale;
+  dim3 grid((T + BQ - 1) / BQ, B * H);
+  dkdv_kernel<<<grid, 192, DKV_SMEM, st>>>(tq, td, lse, Dv, dqkv, T, H, scale, sl2);
+  dq_kernel<<<grid, 192, DQ_SMEM, st>>>(tq, td, lse, Dv, dqkv, T, H, scale, sl2);
+  return cudaGetLastError();
+}
+
+}  // namespace tcfa

@@ -3,6 +3,7 @@
 // one device error word.
 #include "tc_gemm.cu"
 #include "attention_tc.cuh"
+#include "attention_tc_bwd.cuh"
 #include "model_pass.cuh"
 
 #include <mutex>
@@ -295,7 +296,7 @@ int gpt2_attention_backward(const void* qkv, const void* out, const void* dout, 
                             float* work, int B, int T, int H, void* stream) {
   if (!qkv || !out || !dout || !lse || !dqkv || !work || B < 1 || T < 1 || H < 1) return GPT2_EINVAL;
   if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(dqkv)) return GPT2_EINVAL;
-  return attn::flash_backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, work, B, T, H,
+  return tcfa::backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, work, B, T, H,
                               (cudaStream_t)stream) == cudaSuccess
              ? GPT2_OK
              : GPT2_ECUDA;
@@ -338,7 +339,7 @@ int gpt2_attention_backward_noalloc(const void* qkv, const void* out, const void
   if ((long long)B * H * T > (long long)GPT2_ATTN_NOALLOC_MAX_ROWS) return GPT2_EINVAL;
   float* scratch = noalloc_scratch_on_current_device();
   if (scratch == nullptr) return GPT2_ECUDA;
-  return attn::flash_backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, scratch, B, T,
+  return tcfa::backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, scratch, B, T,
                               H, (cudaStream_t)stream) == cudaSuccess
              ? GPT2_OK
              : GPT2_ECUDA;

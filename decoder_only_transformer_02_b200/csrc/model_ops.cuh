@@ -246,7 +246,7 @@ static int op_attn_bwd(gpt2* h, int l) {
   uint8_t* att = h->att + (size_t)l * h->Mmax() * h->C * h->es;
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;
   if (h->prec == GPT2_BF16) {
-    if (attn::flash_backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
+    if (tcfa::backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
                              h->B, h->T, h->H, h->stream) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention backward launch");
     h->launches += 3;
