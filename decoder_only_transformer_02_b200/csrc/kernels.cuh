@@ -351,108 +351,116 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 }
 
 // ------------------------------------------------------- cross-entropy
-// One CTA per row of logits z[M, V] (row kept in shared memory):
+// One CTA per row of logits z[M, V] (the row kept in shared memory):
 //   lse = max + log(sum exp(z - max)); loss_row = lse - z[y]; argmax (lowest
 //   index among maxima).  When write_grad, the row is overwritten in place by
 //   dz = (exp(z - lse) - [j == y]) * gscale.
+// One pass over global memory in and (with write_grad) one out: the load pass
+// keeps a per-thread running (max, argmax, sum of exp) with rescaling per
+// 16-byte chunk, and the gradient pass reads and writes 16-byte chunks.
+// V * sizeof(T) must be a multiple of 16.
+template <typename T>
+__device__ __forceinline__ void ce_combine(float& m, float& s, int& i, float om, float os, int oi) {
+  // merge (m, s, i) with (om, os, oi): max, rescaled sum, lowest argmax
+  const float nm = fmaxf(m, om);
+  const float a = (m == -INFINITY) ? 0.f : __expf(m - nm);
+  const float b = (om == -INFINITY) ? 0.f : __expf(om - nm);
+  s = s * a + os * b;
+  if (om > m || (om == m && oi < i)) i = oi;
+  m = nm;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(1024) ce_kernel(T* __restrict__ z, const int32_t* __restrict__ y, int V,
                                                   float* __restrict__ lse_out, float* __restrict__ loss_row,
                                                   int32_t* __restrict__ amax_out, int write_grad, float gscale) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
-  T* row_s = reinterpret_cast<T*>(sm_raw);
-  __shared__ float red_v[32];
+  uint4* row_s = reinterpret_cast<uint4*>(sm_raw);
+  __shared__ float red_m[32], red_s[32];
   __shared__ int red_i[32];
-  __shared__ float red_s[32];
   const long row = blockIdx.x;
   T* zr = z + row * (long)V;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  // load the row (16-byte chunks) and find max / argmax
   constexpr int EPC = 16 / sizeof(T);
   const int nch = V / EPC;
-  float mx = -INFINITY;
+  float m = -INFINITY, se = 0.f;
   int mi = 0x7fffffff;
   for (int c = tid; c < nch; c += blockDim.x) {
     const uint4 u = reinterpret_cast<const uint4*>(zr)[c];
-    reinterpret_cast<uint4*>(row_s)[c] = u;
+    row_s[c] = u;
     const T* e = reinterpret_cast<const T*>(&u);
+    float v[EPC];
+    float cm = -INFINITY;
+    int ci = 0;
 #pragma unroll
-    for (int i = 0; i < EPC; ++i) {
-      const float v = ld_f(e + i);
-      if (v > mx) {
-        mx = v;
-        mi = c * EPC + i;
+    for (int k = 0; k < EPC; ++k) {
+      v[k] = ld_f(e + k);
+      if (v[k] > cm) {
+        cm = v[k];
+        ci = c * EPC + k;
       }
     }
+    float cs = 0.f;
+#pragma unroll
+    for (int k = 0; k < EPC; ++k) cs += __expf(v[k] - cm);
+    ce_combine<T>(m, se, mi, cm, cs, ci);
   }
-  for (int j = nch * EPC + tid; j < V; j += blockDim.x) {
-    const T v0 = zr[j];
-    row_s[j] = v0;
-    const float v = ld_f(&v0);
-    if (v > mx) {
-      mx = v;
-      mi = j;
-    }
-  }
-  // (max, lowest index) reduction
+  // (max, sum, lowest argmax) across the warp, then across warps
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, mx, o);
+    const float om = __shfl_xor_sync(0xffffffffu, m, o);
+    const float os = __shfl_xor_sync(0xffffffffu, se, o);
     const int oi = __shfl_xor_sync(0xffffffffu, mi, o);
-    if (ov > mx || (ov == mx && oi < mi)) {
-      mx = ov;
-      mi = oi;
-    }
+    ce_combine<T>(m, se, mi, om, os, oi);
   }
   if (lane == 0) {
-    red_v[warp] = mx;
+    red_m[warp] = m;
+    red_s[warp] = se;
     red_i[warp] = mi;
   }
   __syncthreads();
   if (warp == 0) {
-    mx = lane < nw ? red_v[lane] : -INFINITY;
+    m = lane < nw ? red_m[lane] : -INFINITY;
+    se = lane < nw ? red_s[lane] : 0.f;
     mi = lane < nw ? red_i[lane] : 0x7fffffff;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, mx, o);
+      const float om = __shfl_xor_sync(0xffffffffu, m, o);
+      const float os = __shfl_xor_sync(0xffffffffu, se, o);
       const int oi = __shfl_xor_sync(0xffffffffu, mi, o);
-      if (ov > mx || (ov == mx && oi < mi)) {
-        mx = ov;
-        mi = oi;
-      }
+      ce_combine<T>(m, se, mi, om, os, oi);
     }
     if (lane == 0) {
-      red_v[0] = mx;
+      red_m[0] = m;
+      red_s[0] = se;
       red_i[0] = mi;
     }
   }
   __syncthreads();
-  mx = red_v[0];
-  const int amax = red_i[0];
-  // sum of exponentials
-  float se = 0.f;
-  for (int j = tid; j < V; j += blockDim.x) se += __expf(ld_f(row_s + j) - mx);
-  se = warp_sum(se);
-  if (lane == 0) red_s[warp] = se;
-  __syncthreads();
-  if (warp == 0) {
-    se = lane < nw ? red_s[lane] : 0.f;
-    se = warp_sum(se);
-    if (lane == 0) red_s[0] = se;
-  }
-  __syncthreads();
-  const float lse = mx + logf(red_s[0]);
+  const float lse = red_m[0] + logf(red_s[0]);
   const int tgt = y ? y[row] : -1;
   if (tid == 0) {
     if (lse_out) lse_out[row] = lse;
-    if (amax_out) amax_out[row] = amax;
-    if (loss_row) loss_row[row] = (tgt >= 0 && tgt < V) ? lse - ld_f(row_s + tgt) : 0.f;
+    if (amax_out) amax_out[row] = red_i[0];
+    if (loss_row) {
+      float zt = 0.f;
+      if (tgt >= 0 && tgt < V) zt = ld_f(reinterpret_cast<const T*>(row_s) + tgt);
+      loss_row[row] = (tgt >= 0 && tgt < V) ? lse - zt : 0.f;
+    }
   }
   if (write_grad) {
-    for (int j = tid; j < V; j += blockDim.x) {
-      float p = __expf(ld_f(row_s + j) - lse);
-      if (j == tgt) p -= 1.f;
-      st_f(zr + j, p * gscale);
+    for (int c = tid; c < nch; c += blockDim.x) {
+      const uint4 u = row_s[c];
+      const T* e = reinterpret_cast<const T*>(&u);
+      uint4 w;
+      T* o = reinterpret_cast<T*>(&w);
+#pragma unroll
+      for (int k = 0; k < EPC; ++k) {
+        float p = __expf(ld_f(e + k) - lse);
+        if (c * EPC + k == tgt) p -= 1.f;
+        st_f(o + k, p * gscale);
+      }
+      reinterpret_cast<uint4*>(zr)[c] = w;
     }
   }
 }
