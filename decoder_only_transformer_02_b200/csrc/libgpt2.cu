@@ -55,6 +55,12 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_t** out) {
 void gpt2_destroy(gpt2_t* h) {
   if (h == nullptr) return;
   cudaStreamSynchronize(h->stream);
+  if (h->cap_stream) cudaStreamSynchronize(h->cap_stream);
+  for (auto& g : h->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  if (h->ev_in) cudaEventDestroy(h->ev_in);
+  if (h->ev_out) cudaEventDestroy(h->ev_out);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   free_all(h);
   delete h;
@@ -85,8 +91,7 @@ int gpt2_backward(gpt2_t* h, float loss_scale) {
 int gpt2_forward_backward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int B, int T, float loss_scale,
                           float* h_loss) {
   if (h == nullptr) return GPT2_EINVAL;
-  RET_IF(forward_impl(h, tok, tgt, B, T, true, loss_scale));
-  RET_IF(backward_impl(h, loss_scale, true));
+  RET_IF(fused_micro_step(h, tok, tgt, B, T, loss_scale));
   if (h_loss) {
     RET_IF(check_device_flags(h));
     CU_CHECK(h, cudaMemcpy(h_loss, h->d_loss, 4, cudaMemcpyDeviceToHost));
@@ -125,8 +130,7 @@ int gpt2_train_step(gpt2_t* h, const int32_t* h_tok, const int32_t* h_tgt, int n
   for (int k = 0; k < n_micro; ++k) {
     CU_CHECK(h, cudaMemcpyAsync(h->tok_dev, h_tok + k * M, M * 4, cudaMemcpyHostToDevice, h->stream));
     CU_CHECK(h, cudaMemcpyAsync(h->tgt_dev, h_tgt + k * M, M * 4, cudaMemcpyHostToDevice, h->stream));
-    RET_IF(forward_impl(h, h->tok_dev, h->tgt_dev, B, T, true, scale));
-    RET_IF(backward_impl(h, scale, true));
+    RET_IF(fused_micro_step(h, h->tok_dev, h->tgt_dev, B, T, scale));
   }
   RET_IF(adamw_impl(h, lr, wd, b1, b2, eps, clip));
   if (h_loss || h_norm) {
@@ -247,6 +251,12 @@ int gpt2_get_embed_keys(gpt2_t* h, uint32_t* dst) {
 }
 
 int64_t gpt2_kernel_launches(const gpt2_t* h) { return h ? h->launches : -1; }
+
+int gpt2_set_graphs(gpt2_t* h, int enable) {
+  if (h == nullptr) return GPT2_EINVAL;
+  h->use_graphs = enable != 0;
+  return GPT2_OK;
+}
 
 int gpt2_set_timing(gpt2_t* h, int enable) {
   if (h == nullptr) return GPT2_EINVAL;

@@ -79,6 +79,19 @@ struct gpt2 {
   const int32_t* last_tok = nullptr;
   const int32_t* last_tgt = nullptr;
 
+  // CUDA graphs of the fused micro-step, one per (B, T, loss scale)
+  struct GraphEntry {
+    int B, T;
+    uint32_t scale_bits;
+    int state;  // 0: seen once (ran eagerly), 1: captured, -1: capture failed
+    cudaGraphExec_t exec;
+    int64_t nlaunch;
+  };
+  std::vector<GraphEntry> graphs;
+  bool use_graphs = true;
+  cudaStream_t cap_stream = nullptr;
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+
   // opt-in per-class device timing (measurement support)
   bool timing = false;
   std::vector<cudaEvent_t> ev_pool;   // 2 events per timed operation

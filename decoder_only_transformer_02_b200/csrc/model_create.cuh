@@ -181,6 +181,9 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   else
     CU_CHECK(h, cudaFuncSetAttribute(k::ce_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_smem));
   CU_CHECK(h, cudaFuncSetAttribute(k::sort_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, h->sort_cap * 4));
+  CU_CHECK(h, cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+  CU_CHECK(h, cudaEventCreateWithFlags(&h->ev_in, cudaEventDisableTiming));
+  CU_CHECK(h, cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming));
   CU_CHECK(h, cudaStreamSynchronize(h->stream));
   return GPT2_OK;
 }

@@ -186,3 +186,81 @@ static int check_device_flags(gpt2* h) {
   }
   return GPT2_OK;
 }
+
+// One fused micro-step (forward with targets + backward, loss scaled by
+// loss_scale).  The ids are first copied to the handle's private buffers.  With
+// graphs enabled and timing off, the kernel sequence is captured into a CUDA
+// graph the second time a (B, T, loss_scale) combination is seen (the first
+// run is eager and also initialises the kernels' one-time attributes) and
+// replayed afterwards on a private stream joined to the handle's stream with
+// events.  A failed capture falls back to eager launches for that key.
+static int fused_micro_step(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, int T, float loss_scale) {
+  if (tok == nullptr || tgt == nullptr) return set_err(h, GPT2_EINVAL, "fused forward-backward needs ids and targets");
+  if (B < 1 || T < 1 || B > h->maxB || T > h->maxT)
+    return set_err(h, GPT2_EINVAL, "B, T must satisfy 1 <= B <= max_B and 1 <= T <= max_T");
+  const long M = (long)B * T;
+  if (tok != h->tok_dev) CU_CHECK(h, cudaMemcpyAsync(h->tok_dev, tok, M * 4, cudaMemcpyDeviceToDevice, h->stream));
+  if (tgt != h->tgt_dev) CU_CHECK(h, cudaMemcpyAsync(h->tgt_dev, tgt, M * 4, cudaMemcpyDeviceToDevice, h->stream));
+  auto eager = [&]() -> int {
+    RET_IF(forward_impl(h, h->tok_dev, h->tgt_dev, B, T, true, loss_scale));
+    return backward_impl(h, loss_scale, true);
+  };
+  if (!h->use_graphs || h->timing) return eager();
+  uint32_t sb;
+  memcpy(&sb, &loss_scale, 4);
+  gpt2::GraphEntry* e = nullptr;
+  for (auto& g : h->graphs)
+    if (g.B == B && g.T == T && g.scale_bits == sb) e = &g;
+  if (e == nullptr) {
+    h->graphs.push_back(gpt2::GraphEntry{B, T, sb, 0, nullptr, 0});
+    return eager();
+  }
+  if (e->state < 0) return eager();
+  if (e->state == 0) {
+    // capture on the private stream
+    cudaStream_t user = h->stream;
+    CU_CHECK(h, cudaEventRecord(h->ev_in, user));
+    CU_CHECK(h, cudaStreamWaitEvent(h->cap_stream, h->ev_in, 0));
+    CU_CHECK(h, cudaStreamSynchronize(h->cap_stream));
+    if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+      cudaGetLastError();
+      e->state = -1;
+      return eager();
+    }
+    h->stream = h->cap_stream;
+    const int64_t l0 = h->launches;
+    const int r = eager();
+    h->stream = user;
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &graph);
+    cudaGraphExec_t exec = nullptr;
+    if (r != GPT2_OK || ce != cudaSuccess || graph == nullptr ||
+        cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+      cudaGetLastError();
+      if (graph) cudaGraphDestroy(graph);
+      e->state = -1;
+      if (r != GPT2_OK) return r;
+      h->launches = l0;
+      return eager();
+    }
+    cudaGraphDestroy(graph);
+    e->exec = exec;
+    e->nlaunch = h->launches - l0;
+    h->launches = l0;
+    e->state = 1;
+  }
+  CU_CHECK(h, cudaEventRecord(h->ev_in, h->stream));
+  CU_CHECK(h, cudaStreamWaitEvent(h->cap_stream, h->ev_in, 0));
+  CU_CHECK(h, cudaGraphLaunch(e->exec, h->cap_stream));
+  CU_CHECK(h, cudaEventRecord(h->ev_out, h->cap_stream));
+  CU_CHECK(h, cudaStreamWaitEvent(h->stream, h->ev_out, 0));
+  h->launches += e->nlaunch;
+  // the host-side state the replayed sequence implies
+  h->B = B;
+  h->T = T;
+  h->have_fwd = true;
+  h->have_targets = false;
+  h->logits_valid = false;
+  h->have_bwd_keys = true;
+  return GPT2_OK;
+}

@@ -27,7 +27,7 @@ EXPORTED = [
     "gpt2_get_argmax", "gpt2_get_losses", "gpt2_last_loss", "gpt2_get_embed_keys", "gpt2_kernel_launches",
     "gpt2_last_error", "gpt2_attention_forward", "gpt2_attention_backward", "gpt2_attention_workspace_floats",
     "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes", "gpt2_set_timing", "gpt2_get_timing",
-    "gpt2_attention_backward_noalloc",
+    "gpt2_attention_backward_noalloc", "gpt2_set_graphs",
 ]
 ATTN_NOALLOC_MAX_ROWS = 1 << 20
 KCLASSES = ["matmul", "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd", "cross_entropy",
@@ -91,6 +91,7 @@ def load_library():
         "gpt2_set_timing": (I, [P, I]),
         "gpt2_get_timing": (I, [P, P, P, P, P]),
         "gpt2_attention_backward_noalloc": (I, [P, P, P, P, P, I, I, I, P]),
+        "gpt2_set_graphs": (I, [P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -209,6 +210,9 @@ class GPT2:
                                               b1, b2, eps, clip, ctypes.byref(loss) if want else None,
                                               ctypes.byref(norm) if want else None))
         return (loss.value, norm.value) if want else None
+
+    def set_graphs(self, enable: bool):
+        self._check(self._lib.gpt2_set_graphs(self._h, 1 if enable else 0))
 
     # -- measurement support
     def set_timing(self, enable: bool):

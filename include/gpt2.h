@@ -97,6 +97,12 @@ int gpt2_forward_backward(gpt2_t* h, const int32_t* d_tokens, const int32_t* d_t
                           float loss_scale, float* h_loss);
 /* Set every gradient to zero. */
 int gpt2_zero_grad(gpt2_t* h);
+/* CUDA-graph replay of gpt2_forward_backward / gpt2_train_step micro-steps
+ * (default: enabled).  The kernel sequence of a (B, T, loss_scale)
+ * combination is captured the second time it is used and replayed afterwards,
+ * on a private stream ordered after the handle's stream; results are identical
+ * to eager launches.  Never used while timing is enabled. */
+int gpt2_set_graphs(gpt2_t* h, int enable);
 /* Global-norm clip then AdamW ("Let's reproduce GPT-2 (124M)", Key Takeaways:
  * optimization hyperparameters): n = ||g||_2 over all parameters (tied wte
  * once), s = min(1, clip/(n + 1e-6)), g' = s*g; step t += 1;

@@ -153,6 +153,30 @@ def test_bf16_fused_forward_backward_equals_separate():
     np.testing.assert_array_equal(g1, g2)
 
 
+def test_graph_replay_equals_eager_launches():
+    """The fused micro-step is captured into a CUDA graph on the second use of a
+    (B, T, loss scale) and replayed afterwards: the results must be the very
+    bits the eager launches give, for new batches and after a shape change."""
+    runs = {}
+    for graphs in (False, True):
+        G, O, cfg, m = make(BF_CFG, 2, 128, 1, seed=7)
+        m.set_graphs(graphs)
+        seq = [(2, 128, 0), (2, 128, 1), (2, 128, 2), (1, 96, 3), (2, 128, 4), (1, 96, 5), (1, 96, 6)]
+        out = []
+        for B, T, seed in seq:
+            (tok, tgt), = batch("zipf", cfg.vocab_size, B, T, 40 + seed)
+            m.zero_grad()
+            loss = m.forward_backward(dev(tok), dev(tgt), 0.5, want_loss=True)
+            out.append((loss, m.get_grads()))
+        m.adamw_step(6e-4)
+        out.append((0.0, m.get_params()))
+        runs[graphs] = out
+        m.close()
+    for (la, ga), (lb, gb) in zip(runs[False], runs[True]):
+        assert la == lb
+        np.testing.assert_array_equal(ga, gb)
+
+
 def test_bf16_deterministic_step():
     outs = []
     for _ in range(2):
