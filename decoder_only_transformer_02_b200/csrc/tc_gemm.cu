@@ -12,16 +12,18 @@
 // output index is contiguous.)  Both layouts are read straight from global
 // memory by TMA with the 128-byte swizzle; no transposed copy is ever made.
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   warp 0      TMA producer: fills a ring of shared-memory stages (A tile
 //               128x64, B tile BNx64 per stage) and signals an mbarrier.
 //   warp 1      allocates TMEM and issues tcgen05.mma (one thread): 4 MMAs of
 //               128xBNx16 per stage; tcgen05.commit frees the stage and, at the
 //               end of a tile, marks the accumulator ready.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
-//               row), fused math, vectorised global stores.  Two accumulator
-//               buffers in TMEM let the epilogue of tile i overlap the MMAs of
-//               tile i+1.
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
+//               row), fused math, vectorised global stores.  Warps w and w+4
+//               share a TMEM lane quarter and take the two column halves of the
+//               tile, so every SM sub-partition runs two epilogue warps.  Two
+//               accumulator buffers in TMEM let the epilogue of tile i overlap
+//               the MMAs of tile i+1.
 // Every mbarrier wait is bounded (about two seconds); a wait that gives up
 // records an error in g_device_err and the kernel drains its own in-flight
 // copies and MMAs, frees TMEM and returns.
@@ -34,6 +36,8 @@ namespace tcg {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 template <int BN>
@@ -285,7 +289,7 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
 
 // --------------------------------------------------------------- kernel
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                    const Params p) {
   using L = Layout<BN>;
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], EPI_WARPS);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -419,6 +423,8 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    constexpr int CHUNKS = BN / 64 / (EPI_WARPS / 4);  // 64-column chunks per warp
+    const int cbase = ((warp - 2) >> 2) * CHUNKS * 64;  // first column of this warp's half
     uint32_t tc = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tc) {
       int mb, nb, split;
@@ -434,19 +440,19 @@ __global__ void __launch_bounds__(192, 1)
       // 64 accumulator columns per TMEM wait; the buffer is handed back to the
       // MMA warp as soon as its last columns are in registers
 #pragma unroll 1
-      for (int j = 0; j < BN / 64; ++j) {
+      for (int j = 0; j < CHUNKS; ++j) {
         uint32_t r0[32], r1[32];
-        tmem_ld32(tbase + j * 64, r0);
-        tmem_ld32(tbase + j * 64 + 32, r1);
+        tmem_ld32(tbase + cbase + j * 64, r0);
+        tmem_ld32(tbase + cbase + j * 64 + 32, r1);
         tmem_wait_ld();
-        if (j == BN / 64 - 1) {
+        if (j == CHUNKS - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int col0 = nb * BN + j * 64 + h * 32;
+          const int col0 = nb * BN + cbase + j * 64 + h * 32;
           if (row < p.M && col0 < p.N) {
             if (col0 + 32 <= p.N && p.vec32)
               epi_store<true>(p, row, col0, split, h ? r1 : r0);
@@ -532,7 +538,7 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Pa
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  tc_gemm_kernel<BN><<<grid, 192, L::SMEM_BYTES, st>>>(ta, tb, p);
+  tc_gemm_kernel<BN><<<grid, THREADS, L::SMEM_BYTES, st>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
