@@ -10,8 +10,10 @@
 //          read from TMEM; bf16 P written to shared memory in the 128-byte
 //          swizzled K-major layout the MMA reads)
 //   PV_j = P_j V_j        tcgen05.mma, M=128 x N=64 x K=64, fp32 in TMEM
-//   O    = alpha_j (O + PV_{j-1}) in registers (plain O + PV_{j-1} when no
-//          row of the warp changed its maximum), O/l at the end.
+//   O    = alpha_j (O + PV_{j-1}) in registers, O/l at the end.  The
+//          reference maximum m_j is updated lazily (only when a block raises
+//          some row's maximum by more than 2^8), so most blocks need no
+//          rescale: then alpha_j = 1 and O + PV_{j-1} is all that is done.
 // Warp 0 loads Q once and K_j, V_j through a 3-stage TMA ring; warp 1 issues
 // the MMAs (S_{j+1} is computed while the softmax warps work on S_j); warps
 // 2..5 do the softmax (warp w reads TMEM lanes 32*(w%4)..+31).  S and PV are
@@ -63,6 +65,7 @@ constexpr int FP_OFF = FKV_OFF + 2 * F_STAGES * HTILE;  // two P buffers of 128 
 constexpr int FBAR_OFF = FP_OFF + 2 * TILE;
 constexpr int F_SMEM = FBAR_OFF + 256 + 1024;
 constexpr uint32_t F_TMEM_COLS = 256;           // S0 0, S1 64, PV0 128, PV1 192
+constexpr float RESCALE_LOG2 = 8.f;             // lazy-rescale threshold (log2 units)
 
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse, int T,
@@ -241,8 +244,16 @@ __global__ void __launch_bounds__(192, 2)
       for (int e = 8; e < FBKV; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_new = fmaxf(m, mx * sl2);
-      const float alpha = ex2f(m - m_new);
+      // lazy rescaling: the reference maximum m moves only when some row of
+      // the warp sees a block maximum more than 2^RESCALE_LOG2 above it (and
+      // always for the first block).  O, l and P share the reference, so the
+      // result is exact for any choice of it; P stays <= 2^RESCALE_LOG2.
+      const bool rescale = __any_sync(0xffffffffu, mx * sl2 > m + RESCALE_LOG2);
+      float m_new = m, alpha = 1.f;
+      if (rescale) {
+        m_new = fmaxf(m, mx * sl2);
+        alpha = ex2f(m - m_new);
+      }
       // p = 2^(s*sl2 - m_new) (one FFMA + ex2), row sum in 8 chains, bf16 P
       // into shared memory in the swizzled K-major layout
       float rs8[8];
@@ -281,7 +292,7 @@ __global__ void __launch_bounds__(192, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pv_free[pb]);
-        if (__all_sync(0xffffffffu, alpha == 1.f)) {
+        if (!rescale) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             o[i] += __uint_as_float(a0[i]);
