@@ -198,11 +198,34 @@ __global__ void ln_fwd_kernel(const float* __restrict__ x, const float* __restri
 //   linear layer whose output is this residual point).
 // The column accumulators live in shared memory, one private slice per warp
 // (each lane owns its columns: no conflicts, no atomics), which keeps the
-// register count low enough for several CTAs per SM; all loads of a row are
-// issued before its reductions.  Dynamic shared memory: 3 * C * LN_BWD_WARPS floats.
+// register count low enough for two CTAs per SM.  Dynamic shared memory:
+// 3 * C * LN_BWD_WARPS floats.
 constexpr int LN_BWD_WARPS = 4;
 template <int NV, typename TI>
-__global__ void __launch_bounds__(LN_BWD_WARPS * 32, 3) ln_bwd_kernel(const TI* __restrict__ dy, const float* __restrict__ x,
+__device__ __forceinline__ void ln_bwd_load(const TI* __restrict__ dy, const float* __restrict__ x,
+                                            const float* __restrict__ dres, long row, int lane, int accumulate,
+                                            float4 (&xv)[NV], float4 (&dyv)[NV], float4 (&rv)[NV]) {
+  constexpr int C = 128 * NV;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * C) + lane;
+  const float4* dr = reinterpret_cast<const float4*>(dres + row * C) + lane;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    xv[i] = xr[32 * i];
+    if constexpr (sizeof(TI) == 2) {
+      const uint2 u = reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(dy) + row * C)[lane + 32 * i];
+      const float2 a0 = unpack_bf16x2(u.x), a1 = unpack_bf16x2(u.y);
+      dyv[i] = make_float4(a0.x, a0.y, a1.x, a1.y);
+    } else {
+      dyv[i] = (reinterpret_cast<const float4*>(reinterpret_cast<const float*>(dy) + row * C) + lane)[32 * i];
+    }
+    rv[i] = accumulate ? dr[32 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Software-pipelined: the loads of a warp's next row are issued before the
+// reductions of its current row, so two rows per warp are in flight.
+template <int NV, typename TI>
+__global__ void __launch_bounds__(LN_BWD_WARPS * 32, 2) ln_bwd_kernel(const TI* __restrict__ dy, const float* __restrict__ x,
                                                      const float* __restrict__ mean, const float* __restrict__ rstd,
                                                      const float* __restrict__ gam, float* __restrict__ dres,
                                                      bf16* __restrict__ dres_bf, int M, int rows_per_block,
@@ -219,23 +242,25 @@ __global__ void __launch_bounds__(LN_BWD_WARPS * 32, 3) ln_bwd_kernel(const TI* 
   }
   const long r0 = (long)blockIdx.x * rows_per_block;
   const long r1 = min((long)M, r0 + rows_per_block);
-  for (long row = r0 + warp; row < r1; row += LN_BWD_WARPS) {
-    const float mu = mean[row], rs = rstd[row];
-    const float4* xr = reinterpret_cast<const float4*>(x + row * C) + lane;
-    float4* dr = reinterpret_cast<float4*>(dres + row * C) + lane;
-    float4 xv[NV], dyv[NV], rv[NV];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      xv[i] = xr[32 * i];
-      if constexpr (sizeof(TI) == 2) {
-        const uint2 u = reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(dy) + row * C)[lane + 32 * i];
-        const float2 a0 = unpack_bf16x2(u.x), a1 = unpack_bf16x2(u.y);
-        dyv[i] = make_float4(a0.x, a0.y, a1.x, a1.y);
-      } else {
-        dyv[i] = (reinterpret_cast<const float4*>(reinterpret_cast<const float*>(dy) + row * C) + lane)[32 * i];
-      }
-      rv[i] = accumulate ? dr[32 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 xv[NV], dyv[NV], rv[NV];
+  long row = r0 + warp;
+  float mu = 0.f, rs = 0.f;
+  if (row < r1) {
+    ln_bwd_load<NV, TI>(dy, x, dres, row, lane, accumulate, xv, dyv, rv);
+    mu = mean[row];
+    rs = rstd[row];
+  }
+  for (; row < r1; row += LN_BWD_WARPS) {
+    // next row's loads first
+    const long nrow = row + LN_BWD_WARPS;
+    float4 xn[NV], dyn[NV], rn[NV];
+    float mun = 0.f, rsn = 0.f;
+    if (nrow < r1) {
+      ln_bwd_load<NV, TI>(dy, x, dres, nrow, lane, accumulate, xn, dyn, rn);
+      mun = mean[nrow];
+      rsn = rstd[nrow];
     }
+    float4* dr = reinterpret_cast<float4*>(dres + row * C) + lane;
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
@@ -276,6 +301,14 @@ __global__ void __launch_bounds__(LN_BWD_WARPS * 32, 3) ln_bwd_kernel(const TI* 
       acc[C4 + c4] = b;
       acc[2 * C4 + c4] = d;
     }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      xv[i] = xn[i];
+      dyv[i] = dyn[i];
+      rv[i] = rn[i];
+    }
+    mu = mun;
+    rs = rsn;
   }
   __syncthreads();
   // combine the warps' slices in warp order

@@ -205,9 +205,9 @@ static void free_all(gpt2* h) {
     if (p) cudaFree(p);
 }
 
-// rows handled per CTA by the LayerNorm backward: about 4 CTAs per SM
+// rows handled per CTA by the LayerNorm backward: one wave of 2 CTAs per SM
 static int ln_rows_per_block(long M) {
-  long r = (M + 591) / 592;
+  long r = (M + 295) / 296;
   r = (r + 3) / 4 * 4;
   return (int)(r < 4 ? 4 : r);
 }
