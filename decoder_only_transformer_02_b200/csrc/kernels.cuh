@@ -332,8 +332,10 @@ __global__ void __launch_bounds__(256) partials_reduce_kernel(const float* __res
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
   float s = 0.f;
-  if (col < ncols)
+  if (col < ncols) {
+#pragma unroll 8
     for (int b = warp; b < nblk; b += 8) s += part[(long)b * ncols + col];
+  }
   red[warp][lane] = s;
   __syncthreads();
   if (warp == 0 && col < ncols) {
@@ -392,12 +394,18 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 // keeps a per-thread running (max, argmax, sum of exp) with rescaling per
 // 16-byte chunk, and the gradient pass reads and writes 16-byte chunks.
 // V * sizeof(T) must be a multiple of 16.
+constexpr float CE_LOG2E = 1.4426950408889634f;
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 template <typename T>
 __device__ __forceinline__ void ce_combine(float& m, float& s, int& i, float om, float os, int oi) {
   // merge (m, s, i) with (om, os, oi): max, rescaled sum, lowest argmax
   const float nm = fmaxf(m, om);
-  const float a = (m == -INFINITY) ? 0.f : __expf(m - nm);
-  const float b = (om == -INFINITY) ? 0.f : __expf(om - nm);
+  const float a = (m == -INFINITY) ? 0.f : exp2_approx((m - nm) * CE_LOG2E);
+  const float b = (om == -INFINITY) ? 0.f : exp2_approx((om - nm) * CE_LOG2E);
   s = s * a + os * b;
   if (om > m || (om == m && oi < i)) i = oi;
   m = nm;
@@ -434,8 +442,9 @@ __global__ void __launch_bounds__(1024) ce_kernel(T* __restrict__ z, const int32
       }
     }
     float cs = 0.f;
+    const float ncm = -cm * CE_LOG2E;
 #pragma unroll
-    for (int k = 0; k < EPC; ++k) cs += __expf(v[k] - cm);
+    for (int k = 0; k < EPC; ++k) cs += exp2_approx(fmaf(v[k], CE_LOG2E, ncm));
     ce_combine<T>(m, se, mi, cm, cs, ci);
   }
   // (max, sum, lowest argmax) across the warp, then across warps
@@ -482,6 +491,8 @@ __global__ void __launch_bounds__(1024) ce_kernel(T* __restrict__ z, const int32
     }
   }
   if (write_grad) {
+    // gscale * exp(z - lse) = 2^(z*log2(e) + log2(gscale) - lse*log2(e)): one FFMA and one ex2
+    const float off = __log2f(gscale) - lse * CE_LOG2E;
     for (int c = tid; c < nch; c += blockDim.x) {
       const uint4 u = row_s[c];
       const T* e = reinterpret_cast<const T*>(&u);
@@ -489,9 +500,9 @@ __global__ void __launch_bounds__(1024) ce_kernel(T* __restrict__ z, const int32
       T* o = reinterpret_cast<T*>(&w);
 #pragma unroll
       for (int k = 0; k < EPC; ++k) {
-        float p = __expf(ld_f(e + k) - lse);
-        if (c * EPC + k == tgt) p -= 1.f;
-        st_f(o + k, p * gscale);
+        float p = exp2_approx(fmaf(ld_f(e + k), CE_LOG2E, off));
+        if (c * EPC + k == tgt) p -= gscale;
+        st_f(o + k, p);
       }
       reinterpret_cast<uint4*>(zr)[c] = w;
     }
@@ -504,12 +515,12 @@ __global__ void ce_bwd_kernel(T* __restrict__ z, const int32_t* __restrict__ y, 
                               float gscale) {
   const long row = blockIdx.x;
   T* zr = z + row * (long)V;
-  const float L = lse[row];
+  const float off = __log2f(gscale) - lse[row] * CE_LOG2E;  // the same expression as ce_kernel's
   const int tgt = y[row];
   for (int j = threadIdx.x; j < V; j += blockDim.x) {
-    float p = __expf(ld_f(zr + j) - L);
-    if (j == tgt) p -= 1.f;
-    st_f(zr + j, p * gscale);
+    float p = exp2_approx(fmaf(ld_f(zr + j), CE_LOG2E, off));
+    if (j == tgt) p -= gscale;
+    st_f(zr + j, p);
   }
 }
 
