@@ -118,12 +118,22 @@ __global__ void embed_bwd_reduce_kernel(const uint32_t* __restrict__ keys, const
     const uint32_t tokn = keys[s] >> 16;
     if (tokn >= (uint32_t)V) continue;                   // out-of-range id (already flagged)
     if (s > 0 && (keys[s - 1] >> 16) == tokn) continue;  // not a segment start
-    int e = s + 1;
-    while (e < M && (keys[e] >> 16) == tokn) ++e;
+    // segment end: the keys are sorted by token, so binary-search the first
+    // index past s whose token differs
+    int lo = s + 1, hi = M;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((keys[mid] >> 16) == tokn)
+        lo = mid + 1;
+      else
+        hi = mid;
+    }
+    const int e = lo;
     for (int col = threadIdx.x; col < C; col += blockDim.x) {
       float acc = 0.f;
       // run partials start at s and at each chunk boundary inside [s, e)
       acc += part[(long)s * C + col];
+#pragma unroll 4
       for (int cb = (s / EMB_CH + 1) * EMB_CH; cb < e; cb += EMB_CH) acc += part[(long)cb * C + col];
       dwte[(long)tokn * C + col] += acc;
     }
