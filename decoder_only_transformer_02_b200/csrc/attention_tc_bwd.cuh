@@ -1,6 +1,6 @@
 // Causal attention backward on tcgen05 (bf16 operands, fp32 TMEM accumulators).
 //
-// With P = exp(S/sqrt(d) - lse), D_q = sum_d dO_q . O_q (precomputed):
+// With P = exp(S/sqrt(d) - lse), D_q = sum_d dO_q . O_q (computed by dq_kernel):
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dK = dS^T Q / sqrt(d),
 //   dQ = dS K / sqrt(d).
 // Two deterministic kernels (no atomics), in the structure of the forward:
@@ -320,8 +320,8 @@ constexpr uint32_t DQ_TMEM_COLS = 256;                            // S 0, dP 64,
 
 __global__ void __launch_bounds__(192, 2)
     dq_kernel(const __grid_constant__ CUtensorMap tm_qkv64, const __grid_constant__ CUtensorMap tm_do,
-              const float* __restrict__ lse, const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H,
-              float scale, float sl2) {
+              const bf16* __restrict__ out, const float* __restrict__ lse, float* __restrict__ Dv,
+              bf16* __restrict__ dqkv, int T, int H, float scale, float sl2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
@@ -450,9 +450,29 @@ __global__ void __launch_bounds__(192, 2)
     const int q = qb * BQ + r;
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
     const float l2 = q < T ? lse[((long)b * H + h) * T + q] * 1.4426950408889634f : INFINITY;
-    const float dq_ = q < T ? Dv[((long)b * H + h) * T + q] : 0.f;
-    bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
+    // D_q = sum_d dO[q,d] O[q,d] from the dO tile in shared memory and this
+    // query's row of O; written out for dkdv_kernel, which runs next
+    bool ok = mbar_wait(q_full, 0);
+    float dq_ = 0.f;
+    if (ok && q < T) {
+      const bf16* orow = out + ((long)b * T + q) * C + h * HD;
+      const uint8_t* dorow = smem + DQ_DO_OFF;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < HD / 8; ++c) {
+        const uint4 ov = *reinterpret_cast<const uint4*>(orow + 8 * c);
+        const uint4 dv = *reinterpret_cast<const uint4*>(dorow + sw128(r, c));
+        const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w}, d4[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 of = unpack_bf16x2(o4[e]), df = unpack_bf16x2(d4[e]);
+          acc[e] = fmaf(of.x, df.x, fmaf(of.y, df.y, acc[e]));
+        }
+      }
+      dq_ = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      Dv[((long)b * H + h) * T + q] = dq_;
+    }
+    for (int j = 0; ok && j < nblk; ++j) {
       if (!mbar_wait(s_full, j & 1u)) {
         ok = false;
         break;
@@ -515,7 +535,7 @@ __global__ void __launch_bounds__(192, 2)
   }
 }
 
-// D = rowsum(dO * O) (attn::bwd_dot_kernel), then the two kernels above.
+// dq_kernel first (it also writes D = rowsum(dO * O) to Dv), then dkdv_kernel.
 // Dv: caller-provided fp32 scratch of B*H*T elements.
 static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, bf16* dqkv,
                                    float* Dv, int B, int T, int H, cudaStream_t st) {
@@ -536,15 +556,11 @@ static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16*
   if (make_tmap(&tq64, qkv, 3L * C, (long)B * T, 3L * C, 64, 64) != 0) return cudaErrorInvalidValue;
   if (make_tmap(&td, dout, C, (long)B * T, C, 64, 128) != 0) return cudaErrorInvalidValue;
   if (make_tmap(&td64, dout, C, (long)B * T, C, 64, 64) != 0) return cudaErrorInvalidValue;
-  const long rows = (long)B * T * H;
-  int blocks = (int)((rows * 32 + 255) / 256);
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  attn::bwd_dot_kernel<<<blocks, 256, 0, st>>>(out, dout, Dv, B, T, H);
   const float scale = 1.f / sqrtf((float)HD);
   const float sl2 = 1.4426950408889634f * scale;
   dim3 grid((T + BQ - 1) / BQ, B * H);
+  dq_kernel<<<grid, 192, DQ_SMEM, st>>>(tq64, td, out, lse, Dv, dqkv, T, H, scale, sl2);
   dkdv_kernel<<<grid, 192, DKV_SMEM, st>>>(tq64, td64, lse, Dv, dqkv, T, H, scale, sl2);
-  dq_kernel<<<grid, 192, DQ_SMEM, st>>>(tq64, td, lse, Dv, dqkv, T, H, scale, sl2);
   return cudaGetLastError();
 }
 

@@ -49,6 +49,13 @@ def test_attention_small_elementwise(B, T, H):
     got = from_dev(r["dqkv"])
     for k, name in enumerate("qkv"):
         g, ref = got[..., k * C:(k + 1) * C], dqkv_ref[..., k * C:(k + 1) * C]
+        if not np.any(ref):
+            # T = 1: the single key has probability 1, so dS = P (dP - D) and
+            # with it dQ and dK vanish identically; what is left on the device
+            # is the fp32 rounding of dP - D (64-term dot products of N(0,1)
+            # bf16 values), far below this bound
+            assert np.max(np.abs(g)) < 1e-4, name
+            continue
         assert cosine(g, ref) > 0.999, name
         assert rel_max_err(g, ref) < 4e-2, name
 
