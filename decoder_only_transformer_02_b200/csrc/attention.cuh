@@ -14,9 +14,8 @@
 //   dk_j = sum_i ds_ij q_i / sqrt(d)
 //
 // bf16 path (d = 64): the tcgen05 kernels in attention_tc.cuh (forward) and
-// attention_tc_bwd.cuh (backward); this file holds the backward's row-dot
-// preprocess D = rowsum(dO * O).
-// fp32 path: plain per-row kernels (fp32 parity mode, small shapes).
+// attention_tc_bwd.cuh (backward, which also forms D).
+// fp32 path (this file): plain per-row kernels (fp32 parity mode, small shapes).
 #pragma once
 #include "common.cuh"
 
@@ -25,28 +24,6 @@ namespace attn {
 constexpr int HD = 64;   // head dim of the bf16 path
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
-
-// ------------------------------------------------------------ backward
-// D[b,h,t] = sum_d do[b,t,h,d] * o[b,t,h,d]
-__global__ void bwd_dot_kernel(const bf16* __restrict__ o, const bf16* __restrict__ dout, float* __restrict__ Dv,
-                               int B, int T, int H) {
-  const int C = H * HD;
-  const long rows = (long)B * T * H;
-  const int lane = threadIdx.x & 31;
-  for (long w = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5; w < rows;
-       w += ((long)gridDim.x * blockDim.x) >> 5) {
-    const long bt = w / H;
-    const int h = (int)(w % H);
-    const long off = bt * C + h * HD + 2 * lane;
-    const float2 a = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(o + off));
-    const float2 c = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(dout + off));
-    float s = warp_sum(a.x * c.x + a.y * c.y);
-    if (lane == 0) {
-      const long b = bt / T, t = bt % T;
-      Dv[(b * H + h) * T + t] = s;
-    }
-  }
-}
 
 // ------------------------------------------------------------ fp32 path
 // one warp per (b, h, query i): lse_i and o_i

@@ -249,7 +249,7 @@ static int op_attn_bwd(gpt2* h, int l) {
     if (tcfa::backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
                              h->B, h->T, h->H, h->stream) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention backward launch");
-    h->launches += 3;
+    h->launches += 2;
   } else {
     if (attn::naive_backward((const float*)qkv, (const float*)att, (const float*)h->datt, lse, (float*)h->dqkv,
                              h->attn_D, h->B, h->T, h->H, h->C / h->H, h->stream) != cudaSuccess)
