@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 #pragma unroll
   for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
   if (c0 < N) {
-#pragma unroll 4
+#pragma unroll 8
     for (int r = r0 + rl; r < r1; r += 8) {
       const uint4 u = *reinterpret_cast<const uint4*>(a + (long)r * N + c0);
       const T* e = reinterpret_cast<const T*>(&u);
