@@ -201,6 +201,9 @@ def run_ours(args):
     from decoder_only_transformer_02_b200 import synthetic as S
 
     B, T, accum = WORKLOADS[args.workload]
+    if args.B or args.accum:
+        # a smaller case of the same step (profiling captures only; not a bench line)
+        B, accum = args.B or B, args.accum or accum
     tok_per_step = B * T * accum
     stream = torch.cuda.current_stream()
     m = G.GPT2(G.GPT2Config(L, 12, C, V, VP, 1024, B, T, G.GPT2_BF16), seed=1234 + rank, stream=stream)
@@ -318,7 +321,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Zipf 1.1 token streams)",
-        "config": workload_config(args.workload),
+        "config": workload_config(args.workload) if not (args.B or args.accum) else
+        {"workload": f"smaller profiling case B={B} x T={T} x {accum} (not the benchmark workload)"},
         "mfu": mfu, "mfu_sustained_peak": mfu_sus,
         "flops_per_token": fpt, "flops_convention": "6N + 6*L*T*C (causal attention, halved score count)",
         "mfu_noncausal": value * (fpt + 6.0 * L * T * C) / (world * peaks["bf16_tflops"] * 1e12),
@@ -326,15 +330,113 @@ def run_ours(args):
         "final_loss": loss, "roofline": roofline, "kernels": per_step, "e2e": e2e, "clocks": clk,
         "gpu_launches": launches, "micro_step_launch": "CUDA graph replay (captured on second use)",
     }
+    m.close()
+    if world == 1 and not (args.B or args.accum) and not args.no_sub_records:
+        del d_tok, d_tgt
+        torch.cuda.empty_cache()
+        subs = {}
+        if args.workload == "t1024":
+            subs["t512"] = sub_record_workload(G, S, torch, "t512", peaks)
+        subs["attention"] = sub_record_attention(G, torch, peaks)
+        line["sub_records"] = subs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(B, T, accum)
-    m.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------------------ sub-records
+
+def sub_record_workload(G, S, torch, name, peaks, steps=3, warmup=3):
+    """The same optimizer step on another workload of the pages (one GPU):
+    tokens/s, MFU and per-class device times, timed like the headline."""
+    B, T, accum = WORKLOADS[name]
+    tok_per_step = B * T * accum
+    stream = torch.cuda.current_stream()
+    m = G.GPT2(G.GPT2Config(L, 12, C, V, VP, 1024, B, T, G.GPT2_BF16), seed=4321, stream=stream)
+    n = warmup + steps
+    toks = np.empty((n, accum, B, T), dtype=np.int32)
+    tgts = np.empty_like(toks)
+    for s in range(n):
+        ids = S.zipf_stream(tok_per_step + 1, V, 1.1, seed=5000 + s)
+        for k, (x, y) in enumerate(S.micro_batches(ids, B, T, accum)):
+            toks[s, k], tgts[s, k] = x, y
+    d_tok, d_tgt = torch.from_numpy(toks).cuda(), torch.from_numpy(tgts).cuda()
+
+    def step(s):
+        m.zero_grad()
+        for k in range(accum):
+            m.forward_backward(d_tok[s, k], d_tgt[s, k], 1.0 / accum)
+        m.adamw_step(G.lr_at(1000 + s))
+
+    for s in range(warmup):
+        step(s)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(warmup, n):
+        step(s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    m.set_timing(True)
+    m.get_timing()
+    step(warmup)
+    timing = m.get_timing()
+    m.set_timing(False)
+    m.close()
+    value = tok_per_step / (ms / 1e3)
+    return {"config": workload_config(name), "value": value, "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "warmup": warmup, "mfu": value * flops_per_token(T) / (peaks["bf16_tflops"] * 1e12),
+            "kernels_ms_per_step": {k: d["ms"] for k, d in timing.items() if d["ops"]}}
+
+
+def sub_record_attention(G, torch, peaks, reps=5):
+    """The standalone causal attention workload: B=8, H=12, d=64, T in
+    {1024, 2048, 4096}, forward and backward timed separately with CUDA events
+    around each call; L2 flushed (256 MB write) before every timed call."""
+    from decoder_only_transformer_02_b200.synthetic import normal_array
+    st = torch.cuda.current_stream()
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    out = {"B": 8, "H": 12, "d": 64, "flops_convention": "causal: fwd 2*B*H*T^2*d, bwd 2x fwd",
+           "l2": "flushed before every timed call"}
+    for T in (1024, 2048, 4096):
+        B, H = 8, 12
+        Cc = 64 * H
+        qkv = torch.from_numpy(normal_array((B, T, 3 * Cc), 3)).to(torch.bfloat16).cuda()
+        do = torch.from_numpy(normal_array((B, T, Cc), 4)).to(torch.bfloat16).cuda()
+        o = torch.empty(B, T, Cc, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(B, H, T, dtype=torch.float32, device="cuda")
+        dqkv = torch.empty_like(qkv)
+        wk = torch.empty(G.attention_workspace_floats(B, T, H), dtype=torch.float32, device="cuda")
+        fwd = lambda: G.attention_forward(qkv, o, lse, B, T, H, stream=st)
+        bwd = lambda: G.attention_backward(qkv, o, do, lse, dqkv, wk, B, T, H, stream=st)
+        for _ in range(3):
+            fwd()
+            bwd()
+        G.check_device_error(st)
+        t = {"fwd": 0.0, "bwd": 0.0}
+        for _ in range(reps):
+            for part, call in (("fwd", fwd), ("bwd", bwd)):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                call()
+                e1.record(st)
+                torch.cuda.synchronize()
+                t[part] += e0.elapsed_time(e1) / reps
+        G.check_device_error(st)
+        f = 2.0 * B * H * T * T * 64
+        out[f"T{T}"] = {"fwd_ms": t["fwd"], "bwd_ms": t["bwd"], "fwd_tflops": f / (t["fwd"] / 1e3) / 1e12,
+                        "bwd_tflops": 2 * f / (t["bwd"] / 1e3) / 1e12,
+                        "fwd_frac_of_burst_peak": f / (t["fwd"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                        "bwd_frac_of_burst_peak": 2 * f / (t["bwd"] / 1e3) / 1e12 / peaks["bf16_tflops"]}
+        del qkv, do, o, lse, dqkv, wk
+    return out
 
 
 # ------------------------------------------------------- standalone operators
@@ -411,6 +513,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="t1024")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-records", action="store_true", help="skip the t512 and attention sub-records")
+    ap.add_argument("--B", type=int, default=0, help="override the micro-batch (small profiling cases only)")
+    ap.add_argument("--accum", type=int, default=0, help="override the micro-steps (small profiling cases only)")
     args = ap.parse_args()
     if args.op:
         return run_op(args)

@@ -1,23 +1,24 @@
 // Causal attention on the 5th-generation tensor cores (tcgen05): the forward
-// kernel and the constants and helpers the backward kernels share.
+// kernel and the helpers the backward kernels share.
 //
 // bf16 qkv [B, T, 3C] (q, k, v column blocks, head h in columns h*64..),
 // head dim 64; output o [B, T, C] bf16 and lse [B, H, T] fp32.  One CTA owns
-// 128 queries of one (batch, head) and walks the key blocks of 64 keys up to
-// its last query:
-//   S_j  = Q K_j^T        tcgen05.mma, M=128 x N=64 x K=64, fp32 in TMEM
-//   P_j  = exp(S_j/sqrt(d) - m_j)  (online softmax, one thread per query row,
-//          read from TMEM; bf16 P written to shared memory in the 128-byte
-//          swizzled K-major layout the MMA reads)
-//   PV_j = P_j V_j        tcgen05.mma, M=128 x N=64 x K=64, fp32 in TMEM
-//   O    = alpha_j (O + PV_{j-1}) in registers, O/l at the end.  The
-//          reference maximum m_j is updated lazily (only when a block raises
-//          some row's maximum by more than 2^8), so most blocks need no
-//          rescale: then alpha_j = 1 and O + PV_{j-1} is all that is done.
-// Warp 0 loads Q once and K_j, V_j through a 3-stage TMA ring; warp 1 issues
-// the MMAs (S_{j+1} is computed while the softmax warps work on S_j); warps
-// 2..5 do the softmax (warp w reads TMEM lanes 32*(w%4)..+31).  S and PV are
-// double-buffered in TMEM.  All waits are bounded.
+// 128 queries of one (batch, head) and walks the blocks of 128 keys up to its
+// last query:
+//   S_j  = Q K_j^T        tcgen05.mma, M=128 x N=128 x K=64, fp32 in TMEM
+//   P_j  = exp(S_j/sqrt(d) - m)   (online softmax, one thread per query row
+//          holding the row's 128 scores; bf16 P written back into TMEM)
+//   O   += P_j V_j        tcgen05.mma with A = P_j read from TMEM (K = 128
+//          keys), B = V_j from shared memory; O accumulates in TMEM.
+// The reference maximum m of a row moves lazily: only when a block raises some
+// row's maximum by more than 2^8 (and for the first block).  Then O is
+// rescaled in TMEM (load, multiply, store) before the block's PV MMA; most
+// blocks need no rescale.  O/l at the end.
+// Warp 0 loads Q once and K_j, V_j through a 2-stage TMA ring, warp 1 issues
+// the MMAs (S_{j+1} runs while the softmax warps work on S_j), warps 2..5 do
+// the softmax (warp w reads TMEM lanes 32*(w%4)..+31).  A CTA needs 256 TMEM
+// columns and ~82 KB of shared memory, so two CTAs share an SM and each SM
+// sub-partition runs two softmax warps.  All waits are bounded.
 #pragma once
 #include "common.cuh"
 
@@ -25,17 +26,10 @@ namespace tcfa {
 
 using namespace tcg;
 
-constexpr int BQ = 128;       // queries per CTA
-constexpr int BKV = 128;      // keys per block
-constexpr int HD = 64;        // head dim
-constexpr int KV_STAGES = 3;
+constexpr int BQ = 128;                     // queries per CTA
+constexpr int BKV = 128;                    // keys per block
+constexpr int HD = 64;                      // head dim
 constexpr int TILE = 128 * 64 * 2;          // one 128 x 64 bf16 tile (16 KB)
-constexpr int Q_OFF = 0;
-constexpr int KV_OFF = TILE;                // stage s: K at +2s*TILE, V at +(2s+1)*TILE
-constexpr int P_OFF = KV_OFF + 2 * KV_STAGES * TILE;  // two P buffers of 2 tiles each
-constexpr int BAR_OFF = P_OFF + 4 * TILE;
-constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
-constexpr uint32_t TMEM_COLS = 512;         // S0 0, S1 128, PV0 256, PV1 320
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -51,21 +45,79 @@ __device__ __forceinline__ uint32_t sw128(int r, int chunk) {
   return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4));
 }
 
+// bf16 kind::f16 instruction descriptor: fp32 accumulate, M=128, N given, B
+// K-major (b_mn = 0) or MN-major (b_mn = 1); A K-major (shared memory or TMEM)
+__host__ __device__ constexpr uint32_t att_idesc(int n, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(128 >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]  (A: 128 lanes x 16 bf16 = 8 columns per MMA)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 64 consecutive fp32 TMEM columns of this thread's lane (two loads, no wait)
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+}
+// Bounded wait by every lane of a warp, with a warp-uniform outcome: the warp
+// goes on only if every lane saw the phase complete, so the warp-collective
+// tcgen05.ld / tcgen05.st that follow never run on part of a warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+// Transposing warp reduction: lane L holds v[0..31] (one row, 32 columns);
+// returns to lane L the sum over the 32 lanes of column L, in a fixed order.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = up ? v[i] : v[i + w];
+      const float keep = up ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
+// 1-D bulk copy global -> shared, completing on an mbarrier (16-byte aligned, size % 16 == 0)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- forward
-// The forward walks 64-key blocks so that one CTA needs 256 TMEM columns and
-// about 97 KB of shared memory: two CTAs share an SM, and every SM
-// sub-partition runs two softmax warps, one CTA's softmax overlapping the
-// other's MMAs.
-constexpr int FBKV = 64;                        // keys per block (forward)
-constexpr int F_STAGES = 3;
-constexpr int HTILE = 64 * 64 * 2;              // one 64 x 64 bf16 tile (8 KB)
-constexpr int FQ_OFF = 0;                       // Q: 128 x 64, loaded as two 64-row boxes
-constexpr int FKV_OFF = TILE;                   // stage s: K at +2s*HTILE, V at +(2s+1)*HTILE
-constexpr int FP_OFF = FKV_OFF + 2 * F_STAGES * HTILE;  // two P buffers of 128 x 64 bf16
-constexpr int FBAR_OFF = FP_OFF + 2 * TILE;
+constexpr int F_STAGES = 2;
+constexpr int FQ_OFF = 0;                                 // Q: 128 x 64
+constexpr int FKV_OFF = TILE;                             // stage s: K at +2s*TILE, V at +(2s+1)*TILE
+constexpr int FBAR_OFF = FKV_OFF + 2 * F_STAGES * TILE;
 constexpr int F_SMEM = FBAR_OFF + 256 + 1024;
-constexpr uint32_t F_TMEM_COLS = 256;           // S0 0, S1 64, PV0 128, PV1 192
-constexpr float RESCALE_LOG2 = 8.f;             // lazy-rescale threshold (log2 units)
+constexpr uint32_t F_TMEM_COLS = 256;                     // S [0,128), P (bf16 pairs) [128,192), O [192,256)
+constexpr uint32_t FT_S = 0, FT_P = 128, FT_O = 192;
+constexpr float RESCALE_LOG2 = 8.f;                       // lazy-rescale threshold (log2 units)
 
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse, int T,
@@ -73,15 +125,14 @@ __global__ void __launch_bounds__(192, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FBAR_OFF);
-  uint64_t* q_full = bars;                 // 1
-  uint64_t* kv_full = bars + 1;            // F_STAGES
-  uint64_t* kv_empty = kv_full + F_STAGES;
-  uint64_t* s_full = kv_empty + F_STAGES;  // 2
-  uint64_t* s_free = s_full + 2;           // 2 (count 4)
-  uint64_t* p_full = s_free + 2;           // 2 (count 4)
-  uint64_t* pv_full = p_full + 2;          // 2
-  uint64_t* pv_free = pv_full + 2;         // 2 (count 4)
-  uint64_t* drain = pv_free + 2;
+  uint64_t* q_full = bars;                  // 1
+  uint64_t* kv_full = bars + 1;             // F_STAGES
+  uint64_t* kv_empty = kv_full + F_STAGES;  // F_STAGES
+  uint64_t* s_full = kv_empty + F_STAGES;   // S_j in TMEM
+  uint64_t* s_free = s_full + 1;            // count 4: S_j is in registers
+  uint64_t* p_full = s_free + 1;            // count 4: P_j in TMEM (and O rescaled)
+  uint64_t* pv_done = p_full + 1;           // O += P_j V_j complete
+  uint64_t* drain = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -89,7 +140,7 @@ __global__ void __launch_bounds__(192, 2)
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int C = H * HD;
   const int qlast = min(qb * BQ + BQ - 1, T - 1);  // last query position of the block
-  const int nkv = qlast / FBKV + 1;
+  const int nkv = qlast / BKV + 1;
   const int row0 = b * T;  // first row of this batch in the [B*T, 3C] view
 
   if (threadIdx.x == 0) {
@@ -98,13 +149,10 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_full[i], 1);
-      mbar_init(&pv_free[i], 4);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -122,9 +170,9 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 0) {
     if (lane == 0) {
       // -------------------------------------------------------- producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
       mbar_expect_tx(q_full, TILE);
       tma_load_2d(smem_u32(smem + FQ_OFF), &tm_qkv, h * HD, row0 + qb * BQ, q_full);
-      tma_load_2d(smem_u32(smem + FQ_OFF + HTILE), &tm_qkv, h * HD, row0 + qb * BQ + 64, q_full);
       uint32_t issued = 0;
       for (int j = 0; j < nkv; ++j, ++issued) {
         const int s = j % F_STAGES;
@@ -132,76 +180,62 @@ __global__ void __launch_bounds__(192, 2)
           set_device_err(DERR_WAIT_TIMEOUT);
           break;
         }
-        mbar_expect_tx(&kv_full[s], 2 * HTILE);
-        const uint32_t kd = smem_u32(smem + FKV_OFF + 2 * s * HTILE);
-        tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + j * FBKV, &kv_full[s]);
-        tma_load_2d(kd + HTILE, &tm_qkv, 2 * C + h * HD, row0 + j * FBKV, &kv_full[s]);
+        mbar_expect_tx(&kv_full[s], 2 * TILE);
+        const uint32_t kd = smem_u32(smem + FKV_OFF + 2 * s * TILE);
+        tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + j * BKV, &kv_full[s]);
+        tma_load_2d(kd + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BKV, &kv_full[s]);
       }
-      // drain: every issued K/V load has been consumed by its PV MMA
+      // drain: every issued K/V load has landed before the CTA exits
       for (int s = 0; s < F_STAGES; ++s) {
         if ((uint32_t)s < issued) {
           const uint32_t last = issued - 1 - ((issued - 1 - s) % F_STAGES);
-          if (!mbar_wait(&kv_empty[s], (last / F_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+          if (!mbar_wait_drain(&kv_full[s], (last / F_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
         }
       }
-      if (!mbar_wait(q_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      if (!mbar_wait_drain(q_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer
-      // S: A = Q (K-major), B = K_j (K-major), M=128, N=64
-      const uint32_t id_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(FBKV >> 3) << 17) |
-                            ((uint32_t)(BQ >> 4) << 24);
-      // PV: A = P_j (K-major over keys), B = V_j (MN-major: d contiguous), M=128, N=64
-      const uint32_t id_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(HD >> 3) << 17) |
-                             ((uint32_t)(BQ >> 4) << 24);
+      constexpr uint32_t id_s = att_idesc(BKV, 0);  // S: A = Q, B = K_j, both K-major, N = 128 keys
+      constexpr uint32_t id_pv = att_idesc(HD, 1);  // PV: A = P_j (TMEM), B = V_j MN-major, N = 64
       bool ok = mbar_wait(q_full, 0);
-      tc_fence_after();
       const uint32_t qa = smem_u32(smem + FQ_OFF);
       auto do_pv = [&](int i) -> bool {
-        const int pb = i & 1;
-        if (!mbar_wait(&p_full[pb], (i >> 1) & 1u)) return false;
-        if (i >= 2 && !mbar_wait(&pv_free[pb], ((i - 2) >> 1) & 1u)) return false;
+        if (!mbar_wait(p_full, i & 1u)) return false;
         tc_fence_after();
         const int s = i % F_STAGES;
-        const uint32_t pa = smem_u32(smem + FP_OFF + pb * TILE);
-        const uint32_t va = smem_u32(smem + FKV_OFF + (2 * s + 1) * HTILE);
-        const uint32_t d = tmem + 128 + pb * HD;
+        const uint32_t va = smem_u32(smem + FKV_OFF + (2 * s + 1) * TILE);
 #pragma unroll
-        for (int kk = 0; kk < FBKV / 16; ++kk) {
-          const uint64_t ad = make_sdesc(pa + kk * 32, 0);
-          const uint64_t bd = make_sdesc(va + kk * 2048, 1);
-          tc_mma(d, ad, bd, id_pv, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&pv_full[pb]);
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc_mma_ts(tmem + FT_O, tmem + FT_P + kk * 8, make_sdesc(va + kk * 2048, 1), id_pv,
+                    (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&kv_empty[s]);
+        tc_commit(pv_done);
         return true;
       };
       for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % F_STAGES, sb = j & 1;
+        const int s = j % F_STAGES;
         if (!mbar_wait(&kv_full[s], (j / F_STAGES) & 1u)) {
           ok = false;
           break;
         }
-        if (j >= 2 && !mbar_wait(&s_free[sb], ((j - 2) >> 1) & 1u)) {
+        if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t ka = smem_u32(smem + FKV_OFF + 2 * s * HTILE);
+        const uint32_t ka = smem_u32(smem + FKV_OFF + 2 * s * TILE);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t ad = make_sdesc(qa + kk * 32, 0);
-          const uint64_t bd = make_sdesc(ka + kk * 32, 0);
-          tc_mma(tmem + sb * FBKV, ad, bd, id_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&s_full[sb]);
+        for (int kk = 0; kk < HD / 16; ++kk)
+          tc_mma(tmem + FT_S, make_sdesc(qa + kk * 32, 0), make_sdesc(ka + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+        tc_commit(s_full);
         if (j >= 1 && !do_pv(j - 1)) ok = false;
       }
       if (ok && !do_pv(nkv - 1)) ok = false;
       if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
       tc_commit(drain);
-      if (!mbar_wait(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
     }
   } else {
     // ---------------------------------------------------- softmax warps
@@ -209,31 +243,27 @@ __global__ void __launch_bounds__(192, 2)
     const int r = qw * 32 + lane;           // query row within the block
     const int q = qb * BQ + r;              // query position in the sequence
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
-    float o[HD];
-#pragma unroll
-    for (int i = 0; i < HD; ++i) o[i] = 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (j >> 1) & 1u)) {
+      if (!warp_wait(s_full, j & 1u)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // the 64-key row of S in registers (one TMEM wait), buffer released
-      uint32_t v[FBKV];
-      tmem_ld32(tl + sb * FBKV, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tl + sb * FBKV + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      // the 128-key row of S in registers (one TMEM wait), buffer released
+      uint32_t v[BKV];
+      tmem_ld64(tl + FT_S, v);
+      tmem_ld64(tl + FT_S + 64, v + 64);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      // causal mask on the blocks that reach past the block's first query
-      if (j * FBKV + FBKV - 1 > qb * BQ) {
+      if (lane == 0) mbar_arrive(s_free);
+      // causal mask on the block that reaches past the block's first query
+      if (j * BKV + BKV - 1 > qb * BQ) {
 #pragma unroll
-        for (int e = 0; e < FBKV; ++e)
-          if (j * FBKV + e > q) v[e] = __float_as_uint(-INFINITY);
+        for (int e = 0; e < BKV; ++e)
+          if (j * BKV + e > q) v[e] = __float_as_uint(-INFINITY);
       }
       // row maximum of the raw scores in 8 chains; the positive scale
       // 1/sqrt(d)*log2(e) is applied to the maximum
@@ -241,7 +271,7 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(v[i]);
 #pragma unroll
-      for (int e = 8; e < FBKV; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+      for (int e = 8; e < BKV; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       // lazy rescaling: the reference maximum m moves only when some row of
@@ -254,80 +284,65 @@ __global__ void __launch_bounds__(192, 2)
         m_new = fmaxf(m, mx * sl2);
         alpha = ex2f(m - m_new);
       }
-      // p = 2^(s*sl2 - m_new) (one FFMA + ex2), row sum in 8 chains, bf16 P
-      // into shared memory in the swizzled K-major layout
+      // p = 2^(s*sl2 - m_new) (one FFMA + ex2), row sum in 8 chains, packed
+      // to bf16 pairs in place
       float rs8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
-      uint8_t* pbuf = smem + FP_OFF + sb * TILE;
 #pragma unroll
-      for (int k = 0; k < FBKV / 8; ++k) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = ex2f(fmaf(__uint_as_float(v[8 * k + e]), sl2, -m_new));
-          rs8[e] += pv[e];
-        }
-        const uint4 w = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
-                                   pack_bf16x2(pv[6], pv[7]));
-        *reinterpret_cast<uint4*>(pbuf + sw128(r, k)) = w;
+      for (int e = 0; e < BKV; e += 2) {
+        const float p0 = ex2f(fmaf(__uint_as_float(v[e]), sl2, -m_new));
+        const float p1 = ex2f(fmaf(__uint_as_float(v[e + 1]), sl2, -m_new));
+        rs8[e & 7] += p0;
+        rs8[(e + 1) & 7] += p1;
+        v[e >> 1] = pack_bf16x2(p0, p1);
       }
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
       l = l * alpha + rs;
       m = m_new;
+      // O += P_{j-1} V_{j-1} is complete: the P buffer is free and O final up
+      // to block j-1; rescale O in TMEM when the reference moved
       if (j >= 1) {
-        const int pb = (j - 1) & 1;
-        if (!mbar_wait(&pv_full[pb], ((j - 1) >> 1) & 1u)) {
+        if (!warp_wait(pv_done, (j - 1) & 1u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t a0[32], a1[32];
-        tmem_ld32(tl + 128 + pb * HD, a0);
-        tmem_ld32(tl + 128 + pb * HD + 32, a1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pv_free[pb]);
-        if (!rescale) {
+        if (rescale) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            o[i] += __uint_as_float(a0[i]);
-            o[32 + i] += __uint_as_float(a1[i]);
-          }
-        } else {
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            tmem_ld32(tl + FT_O + half * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            o[i] = (o[i] + __uint_as_float(a0[i])) * alpha;
-            o[32 + i] = (o[32 + i] + __uint_as_float(a1[i])) * alpha;
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tl + FT_O + half * 32, o);
           }
         }
       }
+      tmem_st32(tl + FT_P, v);
+      tmem_st32(tl + FT_P + 32, v + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
     }
     if (ok) {
-      const int pb = (nkv - 1) & 1;
-      if (mbar_wait(&pv_full[pb], ((nkv - 1) >> 1) & 1u)) {
+      if (warp_wait(pv_done, (nkv - 1) & 1u)) {
         tc_fence_after();
-        uint32_t a0[32], a1[32];
-        tmem_ld32(tl + 128 + pb * HD, a0);
-        tmem_ld32(tl + 128 + pb * HD + 32, a1);
+        uint32_t o[HD];
+        tmem_ld64(tl + FT_O, o);
         tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          o[i] += __uint_as_float(a0[i]);
-          o[32 + i] += __uint_as_float(a1[i]);
-        }
         if (q < T) {
           const float inv = 1.f / l;
           bf16* orow = out + ((long)b * T + q) * C + h * HD;
 #pragma unroll
           for (int i = 0; i < HD; i += 8)
-            *reinterpret_cast<uint4*>(orow + i) =
-                make_uint4(pack_bf16x2(o[i] * inv, o[i + 1] * inv), pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv),
-                           pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv), pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv));
+            *reinterpret_cast<uint4*>(orow + i) = make_uint4(
+                pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv),
+                pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv),
+                pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv),
+                pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv));
           lse[((long)b * H + h) * T + q] = (m + __log2f(l)) * 0.6931471805599453f;
         }
       } else {
@@ -344,17 +359,16 @@ __global__ void __launch_bounds__(192, 2)
 }
 
 static inline cudaError_t forward(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static DeviceOnce once;
+  cudaError_t e = run_once_per_device(once, [] {
+    cudaError_t r = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  if (e != cudaSuccess) return e;
   CUtensorMap tm;
   const int C = H * HD;
-  if (make_tmap(&tm, qkv, 3L * C, (long)B * T, 3L * C, 64, 64) != 0) return cudaErrorInvalidValue;
+  if (make_tmap(&tm, qkv, 3L * C, (long)B * T, 3L * C, 64, BKV) != 0) return cudaErrorInvalidValue;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
   dim3 grid((T + BQ - 1) / BQ, B * H);
   fwd_kernel<<<grid, 192, F_SMEM, st>>>(tm, out, lse, T, H, sl2);

@@ -4,6 +4,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 typedef __nv_bfloat16 bf16;
 
 // Library-wide device error word.  Kernels never trap: a bounded wait that
@@ -20,6 +22,15 @@ enum DeviceErr : int {
 __device__ int g_device_err = 0;
 
 __device__ __forceinline__ void set_device_err(int code) { atomicCAS(&g_device_err, 0, code); }
+
+// Time after which a pipeline wait (a warp waiting for its producer or
+// consumer) gives up, in nanoseconds of %globaltimer.  Settable from the host
+// (gpt2_set_wait_limit_ns) so that the give-up path can be exercised; the
+// waits that drain a kernel's own in-flight copies and MMAs before it exits
+// keep the fixed DRAIN_LIMIT_NS instead.
+constexpr unsigned long long DEFAULT_WAIT_LIMIT_NS = 2000000000ull;
+constexpr unsigned long long DRAIN_LIMIT_NS = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = DEFAULT_WAIT_LIMIT_NS;
 
 // --------------------------------------------------------------- numerics
 __device__ __forceinline__ float bf2f(bf16 x) { return __bfloat162float(x); }
@@ -69,6 +80,25 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Softmax-statistics merge: (m, s, i) <- (m, s, i) (+) (om, os, oi), where m is
+// a maximum, s = sum of exp(z - m) and i the lowest index attaining m.  The
+// same fixed merge serves the GEMM epilogue's per-tile partials and the
+// cross-entropy kernels' reductions.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float LOG2E_F = 1.4426950408889634f;
+__device__ __forceinline__ void softmax_stats_merge(float& m, float& s, int& i, float om, float os, int oi) {
+  const float nm = fmaxf(m, om);
+  const float a = (m == -INFINITY) ? 0.f : ex2_approx((m - nm) * LOG2E_F);
+  const float b = (om == -INFINITY) ? 0.f : ex2_approx((om - nm) * LOG2E_F);
+  s = s * a + os * b;
+  if (om > m || (om == m && oi < i)) i = oi;
+  m = nm;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -76,3 +106,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 static inline int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
+
+// Host-side set-up that must run once on every device a kernel is launched on
+// (cudaFuncSetAttribute applies to the current device only).
+struct DeviceOnce {
+  std::mutex mu;
+  bool done[64] = {};
+};
+template <class F>
+static cudaError_t run_once_per_device(DeviceOnce& once, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(once.mu);
+  if (once.done[dev]) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess) once.done[dev] = true;
+  return e;
+}

@@ -519,6 +519,88 @@ __global__ void __launch_bounds__(1024) ce_kernel(T* __restrict__ z, const int32
   }
 }
 
+// Cross-entropy from the lm_head GEMM's softmax statistics (bf16 mode).  The
+// GEMM epilogue stored the bf16 logits z[M, V] and, per row and half tile of
+// 128 columns, (max, sum of exp(z - max), lowest argmax) of the stored values.
+// One CTA per row merges the row's partials in a fixed order:
+//   lse = max + log(sum);  loss_row = lse - z[y];  argmax (lowest index)
+// and, when write_grad, streams the row once, overwriting it in place with
+//   dz = (exp(z - lse) - [j == y]) * gscale.
+// V must be a multiple of 8.
+constexpr int CEF_THREADS = 256;
+__global__ void __launch_bounds__(CEF_THREADS) ce_finish_kernel(bf16* __restrict__ z, const float* __restrict__ part,
+                                                               int nh, const int32_t* __restrict__ y, int V,
+                                                               float* __restrict__ lse_out,
+                                                               float* __restrict__ loss_row,
+                                                               int32_t* __restrict__ amax_out, int write_grad,
+                                                               float gscale) {
+  __shared__ float red_m[CEF_THREADS / 32], red_s[CEF_THREADS / 32];
+  __shared__ int red_i[CEF_THREADS / 32];
+  const long row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float m = -INFINITY, s = 0.f;
+  int mi = 0x7fffffff;
+  const float* pr = part + row * (long)nh * 3;
+  for (int k = tid; k < nh; k += CEF_THREADS)
+    softmax_stats_merge(m, s, mi, pr[3 * k], pr[3 * k + 1], __float_as_int(pr[3 * k + 2]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, o);
+    const float os = __shfl_xor_sync(0xffffffffu, s, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, mi, o);
+    softmax_stats_merge(m, s, mi, om, os, oi);
+  }
+  if (lane == 0) {
+    red_m[warp] = m;
+    red_s[warp] = s;
+    red_i[warp] = mi;
+  }
+  __syncthreads();
+  m = red_m[0];
+  s = red_s[0];
+  mi = red_i[0];
+#pragma unroll
+  for (int w = 1; w < CEF_THREADS / 32; ++w) softmax_stats_merge(m, s, mi, red_m[w], red_s[w], red_i[w]);
+  const float lse = m + logf(s);
+  bf16* zr = z + row * (long)V;
+  const int tgt = y ? y[row] : -1;
+  if (tid == 0) {
+    if (lse_out) lse_out[row] = lse;
+    if (amax_out) amax_out[row] = mi;
+    if (loss_row) loss_row[row] = (tgt >= 0 && tgt < V) ? lse - bf2f(zr[tgt]) : 0.f;
+  }
+  if (!write_grad) return;
+  // every thread read the target logit above (tid 0) before any row chunk is
+  // overwritten: the target's chunk is written by a thread that first syncs
+  __syncthreads();
+  // gscale * exp(z - lse) = 2^(z*log2(e) + log2(gscale) - lse*log2(e)): one FFMA and one ex2
+  const float off = __log2f(gscale) - lse * LOG2E_F;
+  const int nch = V / 8;
+  uint4* zc = reinterpret_cast<uint4*>(zr);
+  for (int c0 = tid; c0 < nch; c0 += 4 * CEF_THREADS) {
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (c0 + k * CEF_THREADS < nch) u[k] = zc[c0 + k * CEF_THREADS];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = c0 + k * CEF_THREADS;
+      if (c >= nch) break;
+      uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack_bf16x2(w[e]);
+        float p0 = ex2_approx(fmaf(f.x, LOG2E_F, off));
+        float p1 = ex2_approx(fmaf(f.y, LOG2E_F, off));
+        if (c * 8 + 2 * e == tgt) p0 -= gscale;
+        if (c * 8 + 2 * e + 1 == tgt) p1 -= gscale;
+        w[e] = pack_bf16x2(p0, p1);
+      }
+      zc[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 // dz = (exp(z - lse) - onehot) * gscale in place, from the saved lse
 template <typename T>
 __global__ void ce_bwd_kernel(T* __restrict__ z, const int32_t* __restrict__ y, const float* __restrict__ lse, int V,

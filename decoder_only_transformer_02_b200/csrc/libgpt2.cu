@@ -11,11 +11,12 @@
 
 static std::string g_null_handle_err = "handle is NULL";
 
-// Scratch of gpt2_attention_backward_noalloc: a fixed device array (one fp32
-// per attention row), so that entry point never allocates.  Host code cannot
+// Scratch of gpt2_attention_backward_noalloc: a fixed device array (two fp32
+// per attention row, rows padded to 128-query blocks), so that entry point
+// never allocates.  Host code cannot
 // use the symbol itself as a device address: the address is looked up once per
 // device, with that device current, and cached.
-static __device__ __align__(256) float g_attn_noalloc_scratch[GPT2_ATTN_NOALLOC_MAX_ROWS];
+static __device__ __align__(256) float g_attn_noalloc_scratch[2 * GPT2_ATTN_NOALLOC_MAX_ROWS];
 static std::mutex g_noalloc_mu;
 static float* g_noalloc_addr[256] = {};
 
@@ -291,21 +292,29 @@ const char* gpt2_last_error(const gpt2_t* h) { return h ? h->err.c_str() : g_nul
 // ------------------------------------------------------------ standalone ops
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// The attention kernels launch one grid row per (batch, head): grid.y = B*H.
+static bool attn_sizes_ok(int B, int T, int H) {
+  return B >= 1 && T >= 1 && H >= 1 && (long)B * H <= 65535L && (long)B * T * 3 * 64 * H < (1L << 31);
+}
+
 int gpt2_attention_forward(const void* qkv, void* out, float* lse, int B, int T, int H, void* stream) {
-  if (!qkv || !out || !lse || B < 1 || T < 1 || H < 1) return GPT2_EINVAL;
+  if (!qkv || !out || !lse || !attn_sizes_ok(B, T, H)) return GPT2_EINVAL;
   if (!aligned16(qkv) || !aligned16(out)) return GPT2_EINVAL;
-  if ((long)B * H > 65535L * 1024) return GPT2_EINVAL;
   return tcfa::forward((const bf16*)qkv, (bf16*)out, lse, B, T, H, (cudaStream_t)stream) == cudaSuccess
              ? GPT2_OK
              : GPT2_ECUDA;
 }
 
-int64_t gpt2_attention_workspace_floats(int B, int T, int H) { return (int64_t)B * T * H; }
+int64_t gpt2_attention_workspace_floats(int B, int T, int H) {
+  if (B < 1 || T < 1 || H < 1) return 0;
+  return (int64_t)tcfa::backward_scratch_floats(B, T, H);
+}
 
 int gpt2_attention_backward(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv,
                             float* work, int B, int T, int H, void* stream) {
-  if (!qkv || !out || !dout || !lse || !dqkv || !work || B < 1 || T < 1 || H < 1) return GPT2_EINVAL;
-  if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(dqkv)) return GPT2_EINVAL;
+  if (!qkv || !out || !dout || !lse || !dqkv || !work || !attn_sizes_ok(B, T, H)) return GPT2_EINVAL;
+  if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(dqkv) || !aligned16(work))
+    return GPT2_EINVAL;
   return tcfa::backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, work, B, T, H,
                               (cudaStream_t)stream) == cudaSuccess
              ? GPT2_OK
@@ -344,15 +353,41 @@ size_t gpt2_matmul_workspace_bytes(int M, int N, int K) { return tcg::splitk_wor
 
 int gpt2_attention_backward_noalloc(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv,
                                     int B, int T, int H, void* stream) {
-  if (!qkv || !out || !dout || !lse || !dqkv || B < 1 || T < 1 || H < 1) return GPT2_EINVAL;
+  if (!qkv || !out || !dout || !lse || !dqkv || !attn_sizes_ok(B, T, H)) return GPT2_EINVAL;
   if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(dqkv)) return GPT2_EINVAL;
-  if ((long long)B * H * T > (long long)GPT2_ATTN_NOALLOC_MAX_ROWS) return GPT2_EINVAL;
+  if (tcfa::backward_scratch_floats(B, T, H) > 2L * GPT2_ATTN_NOALLOC_MAX_ROWS) return GPT2_EINVAL;
   float* scratch = noalloc_scratch_on_current_device();
   if (scratch == nullptr) return GPT2_ECUDA;
   return tcfa::backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, scratch, B, T,
                               H, (cudaStream_t)stream) == cudaSuccess
              ? GPT2_OK
              : GPT2_ECUDA;
+}
+
+int gpt2_check_device_error(void* stream) {
+  const cudaError_t se = cudaStreamSynchronize((cudaStream_t)stream);
+  if (se != cudaSuccess) {
+    cudaGetLastError();
+    return GPT2_ECUDA;
+  }
+  int derr = 0;
+  if (cudaMemcpyFromSymbol(&derr, g_device_err, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return GPT2_ECUDA;
+  }
+  if (derr == 0) return GPT2_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_err, &zero, sizeof(int)) != cudaSuccess) cudaGetLastError();
+  return GPT2_ECUDA;
+}
+
+int gpt2_set_wait_limit_ns(uint64_t limit_ns) {
+  const unsigned long long v = limit_ns == 0 ? DEFAULT_WAIT_LIMIT_NS : (unsigned long long)limit_ns;
+  if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return GPT2_ECUDA;
+  }
+  return GPT2_OK;
 }
 
 }  // extern "C"

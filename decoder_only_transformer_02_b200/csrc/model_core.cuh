@@ -50,6 +50,8 @@ struct gpt2 {
   uint8_t *qkv = nullptr, *att = nullptr, *fcu = nullptr, *fca = nullptr, *lnf = nullptr, *logits = nullptr;
   float *lse = nullptr, *lnf_mean = nullptr, *lnf_rstd = nullptr;
   float *ce_lse = nullptr, *losses = nullptr, *d_loss = nullptr;
+  float* ce_part = nullptr;  // lm_head softmax statistics per (row, 128 columns) (bf16 mode)
+  float* attn_cs = nullptr;  // per-128-row-block column sums of dqkv from the attention backward (bf16 mode)
   int32_t* argmax = nullptr;
 
   // backward scratch
@@ -200,7 +202,7 @@ static void free_all(gpt2* h) {
                   h->ce_lse,  h->losses,  h->d_loss,   h->argmax,   h->dres,     h->dln,      h->attn_D,
                   h->ln_part, h->cs_part, h->dres_bf,  h->dbig,     h->dqkv,     h->datt,     h->splitk_ws,
                   h->emb_keys, h->emb_part, h->normbuf, h->d_step, h->norm_part, h->segs,    h->d_bad,    h->tok_dev,
-                  h->tgt_dev};
+                  h->tgt_dev, h->ce_part, h->attn_cs};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }

@@ -112,6 +112,10 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   ALLOC(h, h->lnf_rstd, (size_t)Mx * 4);
   ALLOC(h, h->logits, (size_t)Mx * h->Vp * es);
   ALLOC(h, h->ce_lse, (size_t)Mx * 4);
+  if (h->prec == GPT2_BF16) {
+    ALLOC(h, h->ce_part, (size_t)Mx * tcg::ce_halves(h->Vp) * 3 * 4);
+    ALLOC(h, h->attn_cs, (size_t)h->maxB * ((h->maxT + 127) / 128) * 3 * C * 4);
+  }
   ALLOC(h, h->losses, (size_t)Mx * 4);
   ALLOC(h, h->d_loss, 16);
   ALLOC(h, h->argmax, (size_t)Mx * 4);
@@ -121,7 +125,12 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   ALLOC(h, h->dbig, (size_t)Mx * 4 * C * es);
   ALLOC(h, h->dqkv, (size_t)Mx * 3 * C * es);
   ALLOC(h, h->datt, (size_t)Mx * C * es);
-  ALLOC(h, h->attn_D, (size_t)Mx * H * 4);
+  {
+    // attention backward scratch: per query, lse*log2(e) and D (bf16 mode, padded
+    // to 128-query blocks), or D alone (fp32 mode); the larger of the two
+    const long nb = tcfa::backward_scratch_floats(h->maxB, h->maxT, H);
+    ALLOC(h, h->attn_D, (size_t)(nb > Mx * H ? nb : Mx * H) * 4);
+  }
   {
     const int rpb = ln_rows_per_block(Mx);
     const long nblk = (Mx + rpb - 1) / rpb;
@@ -176,9 +185,7 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   // (exactly the dynamic shared memory each launch asks for; the opt-in limit
   // covers static plus dynamic shared memory)
   const int ce_smem = (int)((size_t)h->Vp * h->es);
-  if (h->prec == GPT2_BF16)
-    CU_CHECK(h, cudaFuncSetAttribute(k::ce_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_smem));
-  else
+  if (h->prec != GPT2_BF16)
     CU_CHECK(h, cudaFuncSetAttribute(k::ce_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_smem));
   CU_CHECK(h, cudaFuncSetAttribute(k::sort_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, h->sort_cap * 4));
   CU_CHECK(h, cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));

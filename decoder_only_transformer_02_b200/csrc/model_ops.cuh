@@ -124,6 +124,25 @@ static int op_lin_fwd(gpt2* h, const void* X, long M, int K, size_t woff, int N,
   return simt_call(h, a);
 }
 
+// bf16 lm_head with the softmax-statistics epilogue: logits[M, Vp] = xf wte^T
+// and h->ce_part
+static int op_lm_head_ce(gpt2* h, long M) {
+  KTimer kt(h, KC_GEMM, 2.0 * M * h->Vp * h->C, 0.0);
+  tcg::GemmArgs g;
+  g.A = (const bf16*)h->lnf;
+  g.lda = h->C;
+  g.B = h->PBF(h->wte);
+  g.ldb = h->C;
+  g.M = (int)M;
+  g.N = h->Vp;
+  g.K = h->C;
+  g.out = h->logits;
+  g.ldc = h->Vp;
+  g.epi = tcg::EPI_CE_STATS;
+  g.ce_part = h->ce_part;
+  return tc_call(h, g);
+}
+
 enum DgradKind { DG_F32, DG_ACT, DG_DGELU };  // fp32 out / activation-typed out / x gelu'(aux)
 
 // dX[M,Kin] = dY[M,N] W[N,Kin]
@@ -219,6 +238,17 @@ static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
   return GPT2_OK;
 }
 
+// grads[boff .. +3C] += the attention backward's per-block column sums of dqkv
+static int op_attn_bias_reduce(gpt2* h, size_t boff) {
+  KTimer kt(h, KC_OTHER, 0.0, 0.0);
+  const int nblk = h->B * ((h->T + 127) / 128);
+  const int n = 3 * h->C;
+  k::partials_reduce_kernel<<<(n + 31) / 32, 256, 0, h->stream>>>(h->attn_cs, nblk, n, n, h->G32(boff), nullptr,
+                                                                  nullptr);
+  LAUNCH_CHECK(h);
+  return GPT2_OK;
+}
+
 // --------------------------------------------------------------- attention
 static int op_attn_fwd(gpt2* h, int l) {
   KTimer kt(h, KC_ATTN_F, 2.0 * h->B * (double)h->T * h->T * h->C, 0.0);
@@ -247,7 +277,7 @@ static int op_attn_bwd(gpt2* h, int l) {
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;
   if (h->prec == GPT2_BF16) {
     if (tcfa::backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
-                             h->B, h->T, h->H, h->stream) != cudaSuccess)
+                       h->B, h->T, h->H, h->stream, h->attn_cs) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention backward launch");
     h->launches += 2;
   } else {

@@ -60,21 +60,26 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
                       w.res(2 * l + 1)));
   }
   RET_IF(op_ln_fwd(h, w.res(2 * L), h->lnfg, h->lnfb, h->lnf, h->lnf_mean, h->lnf_rstd, M));
-  // tied lm_head: logits = xf wte^T (no bias)
-  RET_IF(op_lin_fwd(h, h->lnf, M, C, h->wte, h->Vp, NO_OFF, LIN_NOBIAS, h->logits, nullptr, nullptr));
-  const size_t smem = (size_t)h->Vp * h->es;
   const float gscale = loss_scale / (float)M;
-  {
-  KTimer kt(h, KC_CE, 0.0, (double)M * h->Vp * h->es * (fuse ? 2 : 1));
-  if (h->prec == GPT2_BF16)
-    k::ce_kernel<bf16><<<(unsigned)M, 1024, smem, h->stream>>>((bf16*)h->logits, dtgt, h->Vp, h->ce_lse,
-                                                                dtgt ? h->losses : nullptr, h->argmax, fuse ? 1 : 0,
-                                                                gscale);
-  else
+  if (h->prec == GPT2_BF16) {
+    // tied lm_head: logits = xf wte^T (no bias); the GEMM epilogue also emits
+    // per-(row, 128-column) softmax statistics of the stored logits, so the
+    // cross-entropy pass only merges them and streams the row once for the
+    // gradient
+    RET_IF(op_lm_head_ce(h, M));
+    KTimer kt(h, KC_CE, 0.0, (double)M * h->Vp * 2 * (fuse ? 2 : 0) + (double)M * tcg::ce_halves(h->Vp) * 12);
+    k::ce_finish_kernel<<<(unsigned)M, k::CEF_THREADS, 0, h->stream>>>(
+        (bf16*)h->logits, h->ce_part, tcg::ce_halves(h->Vp), dtgt, h->Vp, h->ce_lse, dtgt ? h->losses : nullptr,
+        h->argmax, fuse ? 1 : 0, gscale);
+    LAUNCH_CHECK(h);
+  } else {
+    RET_IF(op_lin_fwd(h, h->lnf, M, C, h->wte, h->Vp, NO_OFF, LIN_NOBIAS, h->logits, nullptr, nullptr));
+    const size_t smem = (size_t)h->Vp * h->es;
+    KTimer kt(h, KC_CE, 0.0, (double)M * h->Vp * h->es * (fuse ? 2 : 1));
     k::ce_kernel<float><<<(unsigned)M, 1024, smem, h->stream>>>((float*)h->logits, dtgt, h->Vp, h->ce_lse,
                                                                  dtgt ? h->losses : nullptr, h->argmax, fuse ? 1 : 0,
                                                                  gscale);
-  LAUNCH_CHECK(h);
+    LAUNCH_CHECK(h);
   }
   if (dtgt) {
     KTimer kt(h, KC_OTHER, 0.0, 4.0 * M);
@@ -127,7 +132,10 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
     RET_IF(op_lin_wgrad(h, dres_act, M, C, w.att(l), C, o.projw));
     RET_IF(op_lin_dgrad(h, dres_act, M, C, o.projw, C, DG_ACT, h->datt, nullptr));
     RET_IF(op_attn_bwd(h, l));
-    RET_IF(op_colsum(h, h->dqkv, M, 3 * C, o.attnb));
+    if (h->prec == GPT2_BF16)
+      RET_IF(op_attn_bias_reduce(h, o.attnb));
+    else
+      RET_IF(op_colsum(h, h->dqkv, M, 3 * C, o.attnb));
     RET_IF(op_lin_wgrad(h, h->dqkv, M, 3 * C, w.ln1(l), C, o.attnw));
     RET_IF(op_lin_dgrad(h, h->dqkv, M, 3 * C, o.attnw, C, DG_F32, h->dln, nullptr));
     RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l), w.ln1m(l), w.ln1r(l), o.ln1g, o.ln1b, l > 0 ? h->lo[l - 1].mpb : NO_OFF,

@@ -38,7 +38,6 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 template <int BN>
 struct Layout {
@@ -76,13 +75,26 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
+// Bounded wait for the phase with the given parity to complete: gives up
+// (returns false) after g_wait_limit_ns.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0;; ++i) {
+  const uint64_t t0 = globaltimer_ns();
+  // (mbarrier.try_wait itself suspends the thread for a while before it
+  // reports an incomplete phase, so the clock is read on every retry)
+  for (;;) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 255u) == 255u && globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
+    if (globaltimer_ns() - t0 > *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns)) return false;
+  }
+}
+// The same with the fixed limit, for the waits that drain a kernel's own
+// in-flight TMA copies and MMAs before it exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > DRAIN_LIMIT_NS) return false;
   }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
@@ -287,8 +299,110 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
   }
 }
 
+// Softmax statistics epilogue: the 64 accumulator columns [col0, col0+64) of
+// one row are rounded to bf16 and stored (the logits), and their statistics
+// (maximum, sum of exp(z - max), lowest index of the maximum), computed from
+// the rounded values over the columns below N, are merged into (m, s, mi).
+__device__ __forceinline__ void epi_ce_chunk(const Params& p, int row, int col0, uint32_t (&r)[64], float& m,
+                                             float& s, int& mi) {
+  bf16* o = reinterpret_cast<bf16*>(p.out) + (long)row * p.ldc + col0;
+  float cm = -INFINITY;
+  int ci = 0x7fffffff;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float z = bf2f(f2bf(__uint_as_float(r[i])));
+    r[i] = __float_as_uint(z);
+    if (col0 + i < p.N && z > cm) {
+      cm = z;
+      ci = col0 + i;
+    }
+  }
+  if (col0 + 64 <= p.N && p.vec32) {
+    float v[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[16 * q + i]);
+      st_bf16x16(o + 16 * q, v);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (col0 + i < p.N) o[i] = f2bf(__uint_as_float(r[i]));
+  }
+  if (cm == -INFINITY) return;  // no column below N
+  float cs[4] = {0.f, 0.f, 0.f, 0.f};
+  const float nb = -cm * LOG2E_F;
+#pragma unroll
+  for (int i = 0; i < 64; ++i)
+    if (col0 + i < p.N) cs[i & 3] += ex2_approx(fmaf(__uint_as_float(r[i]), LOG2E_F, nb));
+  softmax_stats_merge(m, s, mi, cm, (cs[0] + cs[1]) + (cs[2] + cs[3]), ci);
+}
+
+// The epilogue of one accumulator tile for one warp: its TMEM lane quarter
+// (rows `row` of the tile, one per lane) and its half of the columns
+// [cbase, cbase + BN/2).  release() hands the accumulator buffer back to the
+// MMA issuer once the warp's last columns are in registers (called by lane 0).
+template <int BN, bool CE, class Release>
+__device__ __forceinline__ void epilogue_tile(const Params& p, int row, int nb, int split, uint32_t tbase, int cbase,
+                                              int whalf, int lane, Release release) {
+  constexpr int CHUNKS = BN / 64 / (EPI_WARPS / 4);  // 64-column chunks per warp
+  if constexpr (CE) {
+    // logits and their per-(row, half tile) softmax statistics
+    float m = -INFINITY, s = 0.f;
+    int mi = 0x7fffffff;
+#pragma unroll 1
+    for (int j = 0; j < CHUNKS; ++j) {
+      uint32_t r[64];
+      tmem_ld32(tbase + cbase + j * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(tbase + cbase + j * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_wait_ld();
+      if (j == CHUNKS - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release();
+      }
+      const int col0 = nb * BN + cbase + j * 64;
+      if (row < p.M && col0 < p.N) epi_ce_chunk(p, row, col0, r, m, s, mi);
+    }
+    if (row < p.M) {
+      float* cp = p.ce_part + ((long)row * p.ce_nh + nb * 2 + whalf) * 3;
+      cp[0] = m;
+      cp[1] = s;
+      cp[2] = __int_as_float(mi);
+    }
+  } else {
+    // 64 accumulator columns per TMEM wait; the buffer is handed back to the
+    // MMA warp as soon as its last columns are in registers
+#pragma unroll 1
+    for (int j = 0; j < CHUNKS; ++j) {
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tbase + cbase + j * 64, r0);
+      tmem_ld32(tbase + cbase + j * 64 + 32, r1);
+      tmem_wait_ld();
+      if (j == CHUNKS - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release();
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col0 = nb * BN + cbase + j * 64 + h * 32;
+        if (row < p.M && col0 < p.N) {
+          if (col0 + 32 <= p.N && p.vec32)
+            epi_store<true>(p, row, col0, split, h ? r1 : r0);
+          else
+            epi_store<false>(p, row, col0, split, h ? r1 : r0);
+        }
+      }
+    }
+  }
+}
+
 // --------------------------------------------------------------- kernel
-template <int BN>
+// CE: the softmax-statistics epilogue (EPI_CE_STATS) in its own instantiation,
+// so that its registers do not weigh on the other epilogues.
+template <int BN, bool CE>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                    const Params p) {
@@ -371,7 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int s = 0; s < L::STAGES; ++s) {
         if ((uint32_t)s < issued) {
           const uint32_t last = issued - 1 - ((issued - 1 - s) % L::STAGES);
-          if (!mbar_wait(&full[s], (last / L::STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+          if (!mbar_wait_drain(&full[s], (last / L::STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
         }
       }
     }
@@ -418,7 +532,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // drain: all MMAs issued by this thread have completed
       tc_commit(drain);
-      if (!mbar_wait(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
     }
   } else {
     // --------------------------------------------------------- epilogue
@@ -437,36 +551,259 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int row = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      // 64 accumulator columns per TMEM wait; the buffer is handed back to the
-      // MMA warp as soon as its last columns are in registers
-#pragma unroll 1
-      for (int j = 0; j < CHUNKS; ++j) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tbase + cbase + j * 64, r0);
-        tmem_ld32(tbase + cbase + j * 64 + 32, r1);
-        tmem_wait_ld();
-        if (j == CHUNKS - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col0 = nb * BN + cbase + j * 64 + h * 32;
-          if (row < p.M && col0 < p.N) {
-            if (col0 + 32 <= p.N && p.vec32)
-              epi_store<true>(p, row, col0, split, h ? r1 : r0);
-            else
-              epi_store<false>(p, row, col0, split, h ? r1 : r0);
-          }
-        }
-      }
+      epilogue_tile<BN, CE>(p, row, nb, split, tbase, cbase, (warp - 2) >> 2, lane,
+                            [&] { mbar_arrive(&tempty[buf]); });
     }
   }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)L::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+
+// ------------------------------------------------------ 2-SM kernel
+// A cluster of two CTAs (one per SM) computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256): CTA r of the pair loads rows
+// [r*128, r*128+128) of the tile's A block and rows [r*128, r*128+128) of its
+// B block (the N half) into the same shared-memory offsets, the leader CTA's
+// MMA thread issues the MMAs for both, and each CTA's TMEM receives its 128
+// rows x 256 columns of the accumulator.  Per SM this halves the shared-memory
+// traffic of the B operand against the 1-SM 128 x 256 tile.
+// Barriers: the leader's full[s] counts the bytes of both CTAs' loads (the
+// peer's TMA loads signal it across the pair); the MMA commits release empty[s]
+// and signal tfull[buf] in both CTAs; both CTAs' epilogue warps arrive on the
+// leader's tempty[buf].
+struct Layout2 {
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = BM * BK * 2;   // this CTA's 128 rows of A
+  static constexpr int B_BYTES = 128 * BK * 2;  // this CTA's 128 rows (N half) of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 512;         // two 256-column accumulators
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory that completes on an mbarrier of
+// either CTA of the pair (bar: shared::cluster address)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+// arrive once on the barrier at this offset in both CTAs of the pair when the
+// MMAs issued so far are complete
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+template <bool CE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    tc_gemm2_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                    const Params p) {
+  using L = Layout2;
+  constexpr int BN = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* empty = full + L::STAGES;
+  uint64_t* tfull = empty + L::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)L::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the pair's barriers are initialised before any cross-CTA arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tma_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tma_b)) : "memory");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < p.total_tiles; tile += ncl) {
+        int mb, nb, split;
+        decode_tile(p, tile, mb, nb, split);
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+        const int m0 = mb * 256 + (int)rank * 128, n0 = nb * 256 + (int)rank * 128;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % L::STAGES;
+          const uint32_t ph = (it / L::STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u)) {
+            set_device_err(DERR_WAIT_TIMEOUT);
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(&full[s], 2 * L::STAGE_BYTES);
+          const uint32_t bar = mapa_rank(smem_u32(&full[s]), 0);
+          const uint32_t a_dst = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_dst = a_dst + L::A_BYTES;
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tma_load_2d_pair(a_dst, &tma_a, k0, m0, bar);
+          } else {
+            tma_load_2d_pair(a_dst, &tma_a, m0, k0, bar);
+            tma_load_2d_pair(a_dst + 8192, &tma_a, m0 + 64, k0, bar);
+          }
+          if (!p.b_mn) {
+            tma_load_2d_pair(b_dst, &tma_b, k0, n0, bar);
+          } else {
+            tma_load_2d_pair(b_dst, &tma_b, n0, k0, bar);
+            tma_load_2d_pair(b_dst + 8192, &tma_b, n0 + 64, k0, bar);
+          }
+        }
+      }
+      // drain: every stage this CTA loaded has been consumed by the pair's
+      // MMAs (so its copies have landed) before the CTA goes on to exit
+      const uint32_t issued = it;
+      for (int s = 0; s < L::STAGES; ++s) {
+        if ((uint32_t)s < issued) {
+          const uint32_t last = issued - 1 - ((issued - 1 - s) % L::STAGES);
+          if (!mbar_wait_drain(&empty[s], ((last / L::STAGES) & 1u))) set_device_err(DERR_WAIT_TIMEOUT);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      // -------------------------------------------- MMA issuer (leader CTA)
+      // kind::f16, bf16 x bf16 -> fp32, M = 256 (the pair), N = 256
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)p.a_mn << 15) |
+                             ((uint32_t)p.b_mn << 16) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < p.total_tiles; tile += ncl, ++tc) {
+        int mb, nb, split;
+        decode_tile(p, tile, mb, nb, split);
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+        const uint32_t buf = tc & 1u;
+        if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1u) ^ 1u)) {
+          set_device_err(DERR_WAIT_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % L::STAGES;
+          const uint32_t ph = (it / L::STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph)) {
+            set_device_err(DERR_WAIT_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + L::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = make_sdesc(a_addr + (p.a_mn ? k * 2048 : k * 32), p.a_mn);
+            const uint64_t bd = make_sdesc(b_addr + (p.b_mn ? k * 2048 : k * 32), p.b_mn);
+            tc_mma_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_both(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit_pair_both(&tfull[buf]);
+      }
+      // drain: all MMAs issued by this thread have completed
+      tc_commit_pair_local(drain);
+      if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    constexpr int CHUNKS = BN / 64 / (EPI_WARPS / 4);
+    const int cbase = ((warp - 2) >> 2) * CHUNKS * 64;
+    uint32_t tc = 0;
+    for (int tile = cid; tile < p.total_tiles; tile += ncl, ++tc) {
+      int mb, nb, split;
+      decode_tile(p, tile, mb, nb, split);
+      const uint32_t buf = tc & 1u;
+      if (!mbar_wait(&tfull[buf], (tc >> 1) & 1u)) {
+        set_device_err(DERR_WAIT_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int row = mb * 256 + (int)rank * 128 + q * 32 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      const uint32_t tempty_leader = mapa_rank(smem_u32(&tempty[buf]), 0);
+      epilogue_tile<BN, CE>(p, row, nb, split, tbase, cbase, (warp - 2) >> 2, lane,
+                            [&] { mbar_arrive_cluster(tempty_leader); });
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while its pair may still use its shared memory or TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"((uint32_t)L::TMEM_COLS)
                  : "memory");
   }
@@ -529,21 +866,43 @@ static int num_sms() {
   return n;
 }
 
-template <int BN>
+template <int BN, bool CE>
 static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid, cudaStream_t st) {
   using L = Layout<BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  tc_gemm_kernel<BN><<<grid, THREADS, L::SMEM_BYTES, st>>>(ta, tb, p);
+  static DeviceOnce once;
+  cudaError_t e = run_once_per_device(once, [] {
+    return cudaFuncSetAttribute(tc_gemm_kernel<BN, CE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
+  tc_gemm_kernel<BN, CE><<<grid, THREADS, L::SMEM_BYTES, st>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
-int choose_splits(int tiles, int kb_total) {
-  const int sms = num_sms();
+template <bool CE>
+static cudaError_t launch2(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid, cudaStream_t st) {
+  static DeviceOnce once;
+  cudaError_t e = run_once_per_device(once, [] {
+    return cudaFuncSetAttribute(tc_gemm2_kernel<CE>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout2::SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
+  tc_gemm2_kernel<CE><<<grid, THREADS, Layout2::SMEM_BYTES, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+// Which kernel serves a shape: the 2-SM pair kernel for N > 128 with more
+// than 128 rows when GPT2_GEMM_2SM=1 is set in the environment, else the 1-SM
+// kernel.
+static bool use_pair_kernel(int M, int N, int bn) {
+  static int mode = -1;
+  if (mode < 0) {
+    const char* e = getenv("GPT2_GEMM_2SM");
+    mode = (e != nullptr && e[0] == '1') ? 1 : 0;
+  }
+  return mode == 1 && bn == 256 && M > BM && N > 128;
+}
+
+int choose_splits(int tiles, int kb_total, int units) {
+  const int sms = units;
   if (tiles >= sms) return 1;
   int best = 1;
   double best_eff = (double)tiles / (double)(((tiles + sms - 1) / sms) * sms);
@@ -562,9 +921,10 @@ int choose_splits(int tiles, int kb_total) {
 size_t splitk_workspace_bytes(int M, int N, int K, int bn) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   if (bn != 128) bn = (N <= 128) ? 128 : 256;
-  const int tiles = ceil_div(M, BM) * ceil_div(N, bn);
+  const bool pair = use_pair_kernel(M, N, bn);
+  const int tiles = pair ? ceil_div(M, 256) * ceil_div(N, 256) : ceil_div(M, BM) * ceil_div(N, bn);
   const int kbt = ceil_div(K, BK);
-  const int s = choose_splits(tiles, kbt);
+  const int s = choose_splits(tiles, kbt, pair ? num_sms() / 2 : num_sms());
   return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
 }
 
@@ -576,6 +936,7 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
       (reinterpret_cast<uintptr_t>(g.out) & 15))
     return -1;
   const int bn = (g.bn == 128 || g.N <= 128) ? 128 : 256;
+  const bool pair = use_pair_kernel(g.M, g.N, bn);
   CUtensorMap ta, tb;
   if (!g.a_mn) {
     if (make_tmap(&ta, g.A, g.K, g.M, g.lda, 64, BM)) return -2;
@@ -583,7 +944,7 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
     if (make_tmap(&ta, g.A, g.M, g.K, g.lda, 64, 64)) return -2;
   }
   if (!g.b_mn) {
-    if (make_tmap(&tb, g.B, g.K, g.N, g.ldb, 64, bn)) return -2;
+    if (make_tmap(&tb, g.B, g.K, g.N, g.ldb, 64, pair ? 128 : bn)) return -2;
   } else {
     if (make_tmap(&tb, g.B, g.N, g.K, g.ldb, 64, 64)) return -2;
   }
@@ -593,7 +954,7 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
   p.K = g.K;
   p.a_mn = g.a_mn;
   p.b_mn = g.b_mn;
-  p.num_m = ceil_div(g.M, BM);
+  p.num_m = pair ? ceil_div(g.M, 256) : ceil_div(g.M, BM);
   p.num_n = ceil_div(g.N, bn);
   p.kb_total = ceil_div(g.K, BK);
   p.epi = g.epi;
@@ -603,10 +964,13 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
   p.out2 = g.out2;
   p.aux = g.aux;
   p.ldc = g.ldc;
+  p.ce_part = g.ce_part;
+  p.ce_nh = ce_halves(g.N);
+  if (g.epi == EPI_CE_STATS && (g.ce_part == nullptr || bn != 256)) return -1;
   {
     // 32-byte vector epilogue: every 32-column chunk of every row (and of the
     // residual / aux / split-K partial buffers) must start on 32 bytes
-    const size_t es = (g.epi == EPI_BF16 || g.epi == EPI_GELU || g.epi == EPI_DGELU) ? 2 : 4;
+    const size_t es = (g.epi == EPI_BF16 || g.epi == EPI_GELU || g.epi == EPI_DGELU || g.epi == EPI_CE_STATS) ? 2 : 4;
     auto al32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31) == 0; };
     bool ok = (g.ldc * (long)es) % 32 == 0 && al32(g.out);
     if (g.epi == EPI_RESID_F32) ok = ok && al32(g.resid);
@@ -617,7 +981,7 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
   }
   int splits = 1;
   if (g.epi == EPI_ACCUM_F32 && g.workspace != nullptr) {
-    splits = choose_splits(p.num_m * p.num_n, p.kb_total);
+    splits = choose_splits(p.num_m * p.num_n, p.kb_total, pair ? num_sms() / 2 : num_sms());
     if (splits > 1 && g.workspace_bytes < (size_t)splits * g.M * g.ldc * sizeof(float)) splits = 1;
   }
   if (splits > 1 && g.ldc != g.N) splits = 1;
@@ -633,8 +997,17 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
     p.splits = 1;
   }
   p.total_tiles = p.num_m * p.num_n * p.splits;
-  const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
-  cudaError_t e = (bn == 128) ? launch<128>(ta, tb, p, grid, st) : launch<256>(ta, tb, p, grid, st);
+  cudaError_t e;
+  if (pair) {
+    // one cluster of two CTAs per pair of SMs, persistent over the tiles
+    const int pairs = p.total_tiles < num_sms() / 2 ? p.total_tiles : num_sms() / 2;
+    e = p.epi == EPI_CE_STATS ? launch2<true>(ta, tb, p, 2 * pairs, st) : launch2<false>(ta, tb, p, 2 * pairs, st);
+  } else {
+    const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
+    e = p.epi == EPI_CE_STATS ? launch<256, true>(ta, tb, p, grid, st)
+        : (bn == 128)         ? launch<128, false>(ta, tb, p, grid, st)
+                              : launch<256, false>(ta, tb, p, grid, st);
+  }
   if (e != cudaSuccess) return -3;
   if (splits > 1) {
     const long n = (long)g.M * g.N;

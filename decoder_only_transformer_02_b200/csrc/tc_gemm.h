@@ -14,6 +14,8 @@ enum Epi : int {
   EPI_DGELU = 4,        // out(bf16)  = acc * gelu_tanh'(aux)
   EPI_ACCUM_F32 = 5,    // out(fp32) += acc   (split-K through `workspace` when given)
   EPI_PARTIAL_F32 = 6,  // internal: split-K partial tiles
+  EPI_CE_STATS = 7,     // internal: out(bf16) = acc, plus per-(row, half tile) softmax statistics of the
+                        // stored (bf16-rounded) values into ce_part
 };
 
 // Logical problem: D[M,N] = sum_k A[m,k] B[n,k].
@@ -38,7 +40,11 @@ struct GemmArgs {
   float* workspace = nullptr;   // split-K scratch for EPI_ACCUM_F32 (may be null)
   size_t workspace_bytes = 0;
   int bn = 0;                   // 0: automatic (256 unless N <= 128), or 128 / 256
+  float* ce_part = nullptr;     // EPI_CE_STATS: [M][ce_halves(N)][3] (max, sum of exp(z - max), argmax bits)
 };
+
+// Number of softmax-statistics partials per row that EPI_CE_STATS writes.
+inline int ce_halves(int N) { return 2 * ((N + 255) / 256); }
 
 struct Params {
   int M, N, K;
@@ -54,12 +60,14 @@ struct Params {
   long ldc;
   float* partial;
   int vec32;  // 1: every 32-column chunk is 32-byte aligned (vector epilogue)
+  float* ce_part;
+  int ce_nh;
 };
 
 // Returns 0 on success, -1 bad arguments, -2 tensor-map encode failure, -3 launch failure.
 int gemm(const GemmArgs& g, cudaStream_t stream);
 // Bytes of split-K scratch that an EPI_ACCUM_F32 call of this shape would use.
 size_t splitk_workspace_bytes(int M, int N, int K, int bn);
-int choose_splits(int tiles, int kb_total);
+int choose_splits(int tiles, int kb_total, int units);
 
 }  // namespace tcg

@@ -27,9 +27,9 @@ EXPORTED = [
     "gpt2_get_argmax", "gpt2_get_losses", "gpt2_last_loss", "gpt2_get_embed_keys", "gpt2_kernel_launches",
     "gpt2_last_error", "gpt2_attention_forward", "gpt2_attention_backward", "gpt2_attention_workspace_floats",
     "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes", "gpt2_set_timing", "gpt2_get_timing",
-    "gpt2_attention_backward_noalloc", "gpt2_set_graphs",
+    "gpt2_attention_backward_noalloc", "gpt2_set_graphs", "gpt2_check_device_error", "gpt2_set_wait_limit_ns",
 ]
-ATTN_NOALLOC_MAX_ROWS = 1 << 20
+ATTN_NOALLOC_MAX_ROWS = 1 << 19  # padded (batch, head, position) rows
 KCLASSES = ["matmul", "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd", "cross_entropy",
             "optimizer", "embedding", "other"]
 
@@ -92,6 +92,8 @@ def load_library():
         "gpt2_get_timing": (I, [P, P, P, P, P]),
         "gpt2_attention_backward_noalloc": (I, [P, P, P, P, P, I, I, I, P]),
         "gpt2_set_graphs": (I, [P, I]),
+        "gpt2_check_device_error": (I, [P]),
+        "gpt2_set_wait_limit_ns": (I, [ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -317,7 +319,7 @@ def attention_backward(qkv, out, dout, lse, dqkv, work, B, T, H, stream=None):
 
 def attention_backward_noalloc(qkv, out, dout, lse, dqkv, B, T, H, stream=None):
     """gpt2_attention_backward with the library's fixed scratch array (no
-    allocation; B*H*T <= ATTN_NOALLOC_MAX_ROWS; calls must not overlap)."""
+    allocation; B*H*ceil(T/128)*128 <= ATTN_NOALLOC_MAX_ROWS; calls must not overlap)."""
     _op_check(load_library().gpt2_attention_backward_noalloc(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse),
                                                              _ptr(dqkv), B, T, H, _stream_ptr(stream)),
               "gpt2_attention_backward_noalloc")
@@ -334,6 +336,17 @@ def matmul_bf16(A, lda, a_mn, Bm, ldb, b_mn, M, N, K, epi, bias=None, resid=None
 
 def matmul_workspace_bytes(M, N, K) -> int:
     return int(load_library().gpt2_matmul_workspace_bytes(M, N, K))
+
+
+def check_device_error(stream=None):
+    """Synchronise `stream`, then read and clear the device's error word:
+    raises GPT2Error (ECUDA) when a kernel gave up on a wait since the last check."""
+    _op_check(load_library().gpt2_check_device_error(_stream_ptr(stream)), "a device-side wait gave up")
+
+
+def set_wait_limit_ns(limit_ns: int):
+    """Testing support: the device-side pipeline wait limit (0 = default 2 s)."""
+    _op_check(load_library().gpt2_set_wait_limit_ns(int(limit_ns)), "gpt2_set_wait_limit_ns")
 
 
 def lr_at(it, max_lr=6e-4, min_lr=6e-5, warmup=715, max_steps=19073) -> float:

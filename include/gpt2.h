@@ -171,11 +171,15 @@ const char* gpt2_last_error(const gpt2_t* h);
  * blocks [0,C), [C,2C), [2C,3C) and head h in columns h*64..h*64+63 of each
  * (C = 64*H).  d_out: [B, T, C] bf16.  d_lse: [B, H, T] fp32 natural-log
  * softmax denominators.  Returns GPT2_EINVAL for non-positive sizes or
- * pointers not 16-byte aligned. */
+ * pointers not 16-byte aligned, and when B*H exceeds 65535 (one grid row
+ * per (batch, head)). */
 int gpt2_attention_forward(const void* d_qkv, void* d_out, float* d_lse, int B, int T, int H, void* cuda_stream);
 /* Backward of gpt2_attention_forward: d_dqkv [B, T, 3C] bf16 receives dq, dk,
  * dv in the same column layout.  d_work: caller-provided fp32 scratch of at
- * least gpt2_attention_workspace_floats(B, T, H) elements (rowwise dO.O). */
+ * least gpt2_attention_workspace_floats(B, T, H) elements, 16-byte aligned
+ * (lse*log2(e) and D = rowsum(dO * O) for every query, in whole blocks of 128
+ * queries: 2*B*H*ceil(T/128)*128 floats).  Deterministic: the same inputs
+ * give the same bits. */
 int gpt2_attention_backward(const void* d_qkv, const void* d_out, const void* d_dout, const float* d_lse,
                             void* d_dqkv, float* d_work, int B, int T, int H, void* cuda_stream);
 int64_t gpt2_attention_workspace_floats(int B, int T, int H);
@@ -196,26 +200,51 @@ int gpt2_matmul_bf16(const void* d_A, int64_t lda, int a_mn, const void* d_B, in
 /* Bytes of d_work with which an epi = 5 call of this shape splits over K. */
 size_t gpt2_matmul_workspace_bytes(int M, int N, int K);
 
+/* ---- device-side errors of the standalone operators ----
+ * The kernels never trap.  A pipeline wait that gives up (a producer or
+ * consumer that did not arrive within the wait limit) records an error code
+ * in a per-device error word and the kernel returns early, leaving its outputs
+ * incomplete.  The model handle's syncing calls read that word themselves; the
+ * standalone operators above (and gpt2_attention_backward_noalloc below) are
+ * asynchronous and do not, so callers check it here:
+ * gpt2_check_device_error synchronises cuda_stream (NULL = legacy default
+ * stream), then reads and clears the error word of the current device.
+ * Returns GPT2_OK when no kernel recorded an error since the last check, and
+ * GPT2_ECUDA when one did (or the synchronisation failed).  The word is shared
+ * by every caller on the device: check before trusting a standalone result. */
+int gpt2_check_device_error(void* cuda_stream);
+/* Testing support: the time after which a device-side pipeline wait gives up,
+ * in nanoseconds (0 restores the default of 2 s), on the current device.  The
+ * waits with which a kernel drains its own in-flight copies and MMAs before
+ * returning keep a fixed 2 s limit, so a shortened limit makes kernels give up
+ * early and return cleanly; it never leaves work in flight. */
+int gpt2_set_wait_limit_ns(uint64_t limit_ns);
+
 /* ---- attention backward without any allocation ----
  * (No counterpart in the paper: this is a calling convenience of this library.)
  * The same computation as gpt2_attention_backward, for callers that cannot
  * call cudaMalloc and have no spare device buffer to hand over as d_work: for
  * example a host framework that plans every byte of device memory ahead of
  * time and forbids allocations outside its planner, or a process that runs
- * with the device memory already fully reserved.  Its scratch (one fp32 per
- * (batch, head, position) row) lives in a fixed array inside the library, of
- * GPT2_ATTN_NOALLOC_MAX_ROWS floats (4 MiB); every GPU that loads the library
- * holds that array until the process exits.
- *  - B*H*T must be at most GPT2_ATTN_NOALLOC_MAX_ROWS, else GPT2_EINVAL and
- *    nothing is enqueued.  Other arguments as for gpt2_attention_backward.
+ * with the device memory already fully reserved.  Its scratch (two fp32 per
+ * (batch, head, position) row, rows padded to whole blocks of 128 positions)
+ * lives in a fixed array inside the library of 2 * GPT2_ATTN_NOALLOC_MAX_ROWS
+ * floats (4 MiB); every GPU that loads the library holds that array until the
+ * process exits.
+ *  - B*H*ceil(T/128)*128 must be at most GPT2_ATTN_NOALLOC_MAX_ROWS and B*H at
+ *    most 65535, else GPT2_EINVAL and nothing is enqueued.  Other arguments as
+ *    for gpt2_attention_backward, whose results it reproduces bit for bit.
+ *  - Like the other standalone operators it is asynchronous: a kernel that
+ *    gave up on a wait is reported by gpt2_check_device_error (above), not by
+ *    this call's return value.
  *  - The first call on each device looks up the array's device address on
  *    that device (with it current); make that first call before any stream
  *    capture.  No call allocates device or host memory.
  *  - All calls share the one array and it keeps the last call's contents; the
- *    kernel overwrites every scratch element it reads, so nothing needs to be
+ *    kernels overwrite every scratch element they read, so nothing needs to be
  *    cleared.  Calls that overlap on the GPU (different streams, or different
  *    host threads on one device) race on the array: serialise them. */
-#define GPT2_ATTN_NOALLOC_MAX_ROWS (1 << 20)
+#define GPT2_ATTN_NOALLOC_MAX_ROWS (1 << 19)
 int gpt2_attention_backward_noalloc(const void* d_qkv, const void* d_out, const void* d_dout, const float* d_lse,
                                     void* d_dqkv, int B, int T, int H, void* cuda_stream);
 

@@ -177,6 +177,59 @@ def test_graph_replay_equals_eager_launches():
         np.testing.assert_array_equal(ga, gb)
 
 
+def test_bf16_accumulated_optimizer_step_matches_oracle():
+    """The accumulated optimizer step in bf16 mode: four micro-steps with
+    distinct batches at loss scale 1/4 (the first eager, the second captured
+    into a CUDA graph, the last two replayed), then the global-norm clip
+    (active: clip 1e-2) and AdamW, against the oracle's train_step arithmetic
+    on the same fp32 master weights and moments.  The moments start from a
+    seeded non-zero state at t = 10, so the update is a smooth function of
+    the gradient (at t = 1 it is lr*sign(g), which no tolerance on g bounds).
+    Bars: |dloss| <= 1e-2, per-tensor gradient cosine >= 0.999 (read before
+    the step), norm within 1%, per-tensor cosine of the update dp >= 0.999."""
+    cfgd = dict(n_layer=2, n_head=4, n_embd=256, vocab_size=500, padded_vocab=512, block_size=256)
+    B, T, n_micro, lr, clip = 2, 128, 4, 6e-4, 1e-2
+    G, O, cfg, m = make(cfgd, B, T, 1, seed=5)
+    flat = O.init_params(cfg, 5).astype(np.float32)
+    m.set_params(flat)
+    mbs = batch("zipf", cfg.vocab_size, B, T, 77, n=n_micro)
+    # oracle: accumulated gradients and mean micro-loss, fp64 on the same weights
+    p64 = flat.astype(np.float64)
+    gref = np.zeros_like(p64)
+    lref = []
+    for tok, tgt in mbs:
+        st = O.forward(p64, cfg, tok, tgt)
+        gref += O.backward(st, 1.0 / n_micro)
+        lref.append(st["loss"])
+    rng = np.random.default_rng(3)
+    sg = np.abs(gref) + np.mean(np.abs(gref))
+    m0 = (rng.standard_normal(p64.size) * sg * clip).astype(np.float32)
+    v0 = ((np.abs(rng.standard_normal(p64.size)) + 0.5) * sg * clip) ** 2
+    v0 = v0.astype(np.float32)
+    t0 = 10
+    m.set_adam_state(m0, v0, t0)
+    m.zero_grad()
+    losses = [m.forward_backward(dev(tok), dev(tgt), 1.0 / n_micro, want_loss=True) for tok, tgt in mbs]
+    g = m.get_grads()
+    norm = m.adamw_step(lr, clip=clip, want_norm=True)
+    p1 = m.get_params()
+    m1, v1, t1 = m.get_adam_state()
+    pr, mr, vr, nr = O.adamw_step(p64, gref, m0.astype(np.float64), v0.astype(np.float64), t0 + 1, lr, cfg,
+                                  max_norm=clip)
+    assert t1 == t0 + 1
+    assert abs(float(np.mean(losses)) - float(np.mean(lref))) <= 1e-2
+    cos = per_tensor(g, gref, cfg, cosine)
+    bad = {k: v for k, v in cos.items() if v < 0.999}
+    assert not bad, bad
+    assert abs(norm - nr) / nr < 1e-2
+    assert nr > 10 * clip  # the clip is active
+    dcos = per_tensor(p1.astype(np.float64) - p64, pr - p64, cfg, cosine)
+    bad = {k: v for k, v in dcos.items() if v < 0.999}
+    assert not bad, bad
+    mcos = per_tensor(m1, mr, cfg, cosine)
+    assert min(mcos.values()) >= 0.999, mcos
+
+
 def test_bf16_deterministic_step():
     outs = []
     for _ in range(2):

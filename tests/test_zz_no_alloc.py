@@ -3,11 +3,13 @@ cannot allocate device memory (its scratch is a fixed array inside the
 library).  Called through the C ABI twice in a row, with different and larger
 inputs the second time so that the array's leftover contents are exercised, and
 compared with the allocating entry point gpt2_attention_backward at the
-attention tests' tolerance.  Kept in a file of its own that collects last."""
+attention tests' tolerance.  Both entry points run the same deterministic
+kernels on the same inputs, so the outputs must be bit-identical.  Kept in a
+file of its own that collects last."""
 import numpy as np
 import pytest
 
-from tests.gpu_util import cosine, from_dev, need_gpu, rel_max_err, to_dev_bf16, torch
+from tests.gpu_util import from_dev, need_gpu, to_dev_bf16, torch
 
 pytestmark = pytest.mark.gpu
 
@@ -35,13 +37,9 @@ def test_noalloc_attention_backward_matches_allocating_entry_point():
         G.attention_backward(qkv, out, do, lse, ref, work, B, T, H)
         got = torch.full((B, T, 3 * C), float("nan"), dtype=torch.bfloat16, device="cuda")
         G.attention_backward_noalloc(qkv, out, do, lse, got, B, T, H)
-        torch.cuda.synchronize()
-        g, r = from_dev(got), from_dev(ref)
-        assert np.all(np.isfinite(g))
-        for k in range(3):
-            gk, rk = g[..., k * C:(k + 1) * C], r[..., k * C:(k + 1) * C]
-            assert cosine(gk, rk) > 0.999
-            assert rel_max_err(gk, rk) < 4e-2
+        G.check_device_error()
+        assert np.all(np.isfinite(from_dev(got)))
+        assert torch.equal(got, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
@@ -53,4 +51,8 @@ def test_noalloc_rejects_sizes_beyond_its_array():
     lse = torch.zeros(16, dtype=torch.float32, device="cuda")
     with pytest.raises(G.GPT2Error) as e:
         G.attention_backward_noalloc(dummy, dummy, dummy, lse, dummy, B, T, H)
+    assert e.value.name == "EINVAL"
+    # B*H beyond one grid row per (batch, head), with B*H*T inside the array
+    with pytest.raises(G.GPT2Error) as e:
+        G.attention_backward_noalloc(dummy, dummy, dummy, lse, dummy, 65536, 1, 1)
     assert e.value.name == "EINVAL"
