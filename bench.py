@@ -457,14 +457,20 @@ def run_op(args):
         a_mn, b_mn = {"fwd": (0, 0), "dgrad": (0, 1), "wgrad": (1, 1)}[args.layout]
         A = torch.from_numpy(normal_array((K, M) if a_mn else (M, K), 1)).to(torch.bfloat16).cuda()
         Bm = torch.from_numpy(normal_array((K, N) if b_mn else (N, K), 2)).to(torch.bfloat16).cuda()
-        epi = 5 if args.layout == "wgrad" else 0
-        o = torch.zeros(M, N, dtype=torch.float32 if epi == 5 else torch.bfloat16, device="cuda")
+        epi = args.epi if args.epi >= 0 else (5 if args.layout == "wgrad" else 0)
+        f32_out = epi in (1, 2, 5)
+        o = torch.zeros(M, N, dtype=torch.float32 if f32_out else torch.bfloat16, device="cuda")
+        o2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda") if epi == 3 else None
+        aux = torch.from_numpy(normal_array((M, N), 5)).to(torch.bfloat16).cuda() if epi == 4 else None
+        resid = torch.from_numpy(normal_array((M, N), 6)).cuda() if epi == 2 else None
+        bias = torch.from_numpy(normal_array((N,), 7)).cuda() if epi in (0, 1, 2, 3) else None
         wsb = G.matmul_workspace_bytes(M, N, K) if epi == 5 else 0
         ws = torch.empty(max(1, wsb // 4), dtype=torch.float32, device="cuda")
-        call = lambda: G.matmul_bf16(A, M if a_mn else K, a_mn, Bm, N if b_mn else K, b_mn, M, N, K, epi, out=o,
-                                     ldc=N, work=ws if wsb else None, work_bytes=wsb, stream=st)
+        call = lambda: G.matmul_bf16(A, M if a_mn else K, a_mn, Bm, N if b_mn else K, b_mn, M, N, K, epi, bias=bias,
+                                     resid=resid, out=o, out2=o2, aux=aux, ldc=N, work=ws if wsb else None,
+                                     work_bytes=wsb, stream=st)
         work = 2.0 * M * N * K
-        out.update(shape=[M, N, K], layout=args.layout, splitk_workspace_bytes=wsb)
+        out.update(shape=[M, N, K], layout=args.layout, epilogue=epi, splitk_workspace_bytes=wsb)
     else:
         B, H, T = 8, 12, args.T
         Cc = 64 * H
@@ -505,6 +511,8 @@ def main():
     ap.add_argument("--op", choices=["matmul", "attention"], default=None)
     ap.add_argument("--shape", default="16384,3072,768")
     ap.add_argument("--layout", choices=["fwd", "dgrad", "wgrad"], default="fwd")
+    ap.add_argument("--epi", type=int, default=-1,
+                    help="matmul epilogue (0 bf16+bias, 1 fp32, 2 fp32 residual, 3 GELU, 4 GELU', 5 accumulate)")
     ap.add_argument("--T", type=int, default=1024)
     ap.add_argument("--part", choices=["fwd", "bwd", "both"], default="both")
     ap.add_argument("--gpus", type=int, default=1)

@@ -39,6 +39,23 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+// 2^x on the FMA and integer pipes, to take part of the exponentials off the
+// MUFU unit without using any other MUFU-pipe instruction (no float/int
+// conversion, no rounding instruction): adding 1.5 * 2^23 rounds x to the
+// nearest integer n in the low mantissa bits, f = x - n lies in [-0.5, 0.5],
+// 2^f comes from a cubic fitted here to minimise the maximum relative error
+// on that interval (7.5e-5, below the 2^-9 rounding of the bf16 values it
+// feeds), and n is shifted into the exponent field.  Results below 2^-125
+// (and x = -inf) give 0, as ex2.approx.ftz flushes those below 2^-126.
+__device__ __forceinline__ float ex2_fma(float x) {
+  const float xc = fmaxf(x, -127.f);
+  const float t = xc + 12582912.f;  // 1.5 * 2^23
+  const float f = xc - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.05517144f, f, 0.24261081f), f, 0.69326099f), f, 0.99992809f);
+  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -125.f ? 0.f : y;
+}
+
 // byte offset of element (r, c) in a 128-row, 64-column bf16 K-major tile with
 // the 128-byte swizzle (16-byte chunk c/8 of row r stored at chunk (c/8)^(r%8))
 __device__ __forceinline__ uint32_t sw128(int r, int chunk) {
@@ -110,41 +127,56 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 }
 
 // ---------------------------------------------------------------- forward
+// Persistent: a CTA takes work items (one 128-query block of one (batch,
+// head)) in a fixed order, longest first, and the pipeline runs across item
+// boundaries: the next item's Q and first K/V blocks load and its first S MMA
+// runs while the softmax warps finish the current item's output.
 constexpr int F_STAGES = 2;
-constexpr int FQ_OFF = 0;                                 // Q: 128 x 64
-constexpr int FKV_OFF = TILE;                             // stage s: K at +2s*TILE, V at +(2s+1)*TILE
+constexpr int FQ_OFF = 0;                                 // two Q buffers of 128 x 64
+constexpr int FKV_OFF = 2 * TILE;                         // stage s: K at +2s*TILE, V at +(2s+1)*TILE
 constexpr int FBAR_OFF = FKV_OFF + 2 * F_STAGES * TILE;
 constexpr int F_SMEM = FBAR_OFF + 256 + 1024;
 constexpr uint32_t F_TMEM_COLS = 256;                     // S [0,128), P (bf16 pairs) [128,192), O [192,256)
 constexpr uint32_t FT_S = 0, FT_P = 128, FT_O = 192;
 constexpr float RESCALE_LOG2 = 8.f;                       // lazy-rescale threshold (log2 units)
+#ifndef EX2_FMA_EVERY
+#define EX2_FMA_EVERY 0  // > 0: one pair of exponentials in EX2_FMA_EVERY through ex2_fma instead of MUFU
+#endif
+
+// The w-th work item in descending order of length: 128-row block index and
+// (batch, head) row of the grid.
+__device__ __forceinline__ void item_desc(int w, int nblk, int BH, int& blk, int& bh) {
+  blk = nblk - 1 - w / BH;
+  bh = w % BH;
+}
 
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse, int T,
-               int H, float sl2) {
+               int H, int BH, float sl2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FBAR_OFF);
-  uint64_t* q_full = bars;                  // 1
-  uint64_t* kv_full = bars + 1;             // F_STAGES
+  uint64_t* q_full = bars;                  // 2
+  uint64_t* q_empty = bars + 2;             // 2: the item's last S MMA has read Q
+  uint64_t* kv_full = bars + 4;             // F_STAGES
   uint64_t* kv_empty = kv_full + F_STAGES;  // F_STAGES
-  uint64_t* s_full = kv_empty + F_STAGES;   // S_j in TMEM
-  uint64_t* s_free = s_full + 1;            // count 4: S_j is in registers
-  uint64_t* p_full = s_free + 1;            // count 4: P_j in TMEM (and O rescaled)
-  uint64_t* pv_done = p_full + 1;           // O += P_j V_j complete
+  uint64_t* s_full = kv_empty + F_STAGES;   // S in TMEM
+  uint64_t* s_free = s_full + 1;            // count 4: S is in registers
+  uint64_t* p_full = s_free + 1;            // count 4: P in TMEM (and O rescaled)
+  uint64_t* pv_done = p_full + 1;           // O += P V complete
   uint64_t* drain = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest blocks first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int nqb = (T + BQ - 1) / BQ;
+  const int nitems = nqb * BH;
   const int C = H * HD;
-  const int qlast = min(qb * BQ + BQ - 1, T - 1);  // last query position of the block
-  const int nkv = qlast / BKV + 1;
-  const int row0 = b * T;  // first row of this batch in the [B*T, 3C] view
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
     for (int s = 0; s < F_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -171,68 +203,99 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0) {
       // -------------------------------------------------------- producer
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
-      mbar_expect_tx(q_full, TILE);
-      tma_load_2d(smem_u32(smem + FQ_OFF), &tm_qkv, h * HD, row0 + qb * BQ, q_full);
-      uint32_t issued = 0;
-      for (int j = 0; j < nkv; ++j, ++issued) {
-        const int s = j % F_STAGES;
-        if (!mbar_wait(&kv_empty[s], ((j / F_STAGES) & 1u) ^ 1u)) {
-          set_device_err(DERR_WAIT_TIMEOUT);
+      uint32_t g = 0, t = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int qb, bh;
+        item_desc(w, nqb, BH, qb, bh);
+        const int b = bh / H, h = bh % H, row0 = b * T;
+        const int nkv = min(qb * BQ + BQ - 1, T - 1) / BKV + 1;
+        const uint32_t qbuf = t & 1u;
+        if (!mbar_wait(&q_empty[qbuf], ((t >> 1) & 1u) ^ 1u)) {
+          ok = false;
           break;
         }
-        mbar_expect_tx(&kv_full[s], 2 * TILE);
-        const uint32_t kd = smem_u32(smem + FKV_OFF + 2 * s * TILE);
-        tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + j * BKV, &kv_full[s]);
-        tma_load_2d(kd + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BKV, &kv_full[s]);
+        mbar_expect_tx(&q_full[qbuf], TILE);
+        tma_load_2d(smem_u32(smem + FQ_OFF + qbuf * TILE), &tm_qkv, h * HD, row0 + qb * BQ, &q_full[qbuf]);
+        for (int j = 0; j < nkv; ++j, ++g) {
+          const int s = g % F_STAGES;
+          if (!mbar_wait(&kv_empty[s], ((g / F_STAGES) & 1u) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&kv_full[s], 2 * TILE);
+          const uint32_t kd = smem_u32(smem + FKV_OFF + 2 * s * TILE);
+          tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + j * BKV, &kv_full[s]);
+          tma_load_2d(kd + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BKV, &kv_full[s]);
+        }
       }
-      // drain: every issued K/V load has landed before the CTA exits
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      // drain: every issued load has landed before the CTA exits
       for (int s = 0; s < F_STAGES; ++s) {
-        if ((uint32_t)s < issued) {
-          const uint32_t last = issued - 1 - ((issued - 1 - s) % F_STAGES);
+        if ((uint32_t)s < g) {
+          const uint32_t last = g - 1 - ((g - 1 - s) % F_STAGES);
           if (!mbar_wait_drain(&kv_full[s], (last / F_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
         }
       }
-      if (!mbar_wait_drain(q_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      for (uint32_t i = 0; i < 2; ++i) {
+        if (i < t) {
+          const uint32_t last = t - 1 - ((t - 1 - i) % 2);
+          if (!mbar_wait_drain(&q_full[i], (last >> 1) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        }
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer
       constexpr uint32_t id_s = att_idesc(BKV, 0);  // S: A = Q, B = K_j, both K-major, N = 128 keys
-      constexpr uint32_t id_pv = att_idesc(HD, 1);  // PV: A = P_j (TMEM), B = V_j MN-major, N = 64
-      bool ok = mbar_wait(q_full, 0);
-      const uint32_t qa = smem_u32(smem + FQ_OFF);
-      auto do_pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1u)) return false;
+      constexpr uint32_t id_pv = att_idesc(HD, 1);  // PV: A = P (TMEM), B = V_j MN-major, N = 64
+      uint32_t g = 0, t = 0;
+      int prev_j = 0;  // block index (within its item) of step g-1
+      bool ok = true;
+      auto do_pv = [&](uint32_t gp, int jp) -> bool {
+        if (!mbar_wait(p_full, gp & 1u)) return false;
         tc_fence_after();
-        const int s = i % F_STAGES;
+        const int s = gp % F_STAGES;
         const uint32_t va = smem_u32(smem + FKV_OFF + (2 * s + 1) * TILE);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
           tc_mma_ts(tmem + FT_O, tmem + FT_P + kk * 8, make_sdesc(va + kk * 2048, 1), id_pv,
-                    (i > 0 || kk > 0) ? 1u : 0u);
+                    (jp > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&kv_empty[s]);
         tc_commit(pv_done);
         return true;
       };
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % F_STAGES;
-        if (!mbar_wait(&kv_full[s], (j / F_STAGES) & 1u)) {
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int qb, bh;
+        item_desc(w, nqb, BH, qb, bh);
+        const int nkv = min(qb * BQ + BQ - 1, T - 1) / BKV + 1;
+        const uint32_t qbuf = t & 1u;
+        if (!mbar_wait(&q_full[qbuf], (t >> 1) & 1u)) {
           ok = false;
           break;
         }
-        if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t ka = smem_u32(smem + FKV_OFF + 2 * s * TILE);
+        const uint32_t qa = smem_u32(smem + FQ_OFF + qbuf * TILE);
+        for (int j = 0; j < nkv; ++j, ++g) {
+          const int s = g % F_STAGES;
+          if (!mbar_wait(&kv_full[s], (g / F_STAGES) & 1u) || (g >= 1 && !mbar_wait(s_free, (g - 1) & 1u))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(smem + FKV_OFF + 2 * s * TILE);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          tc_mma(tmem + FT_S, make_sdesc(qa + kk * 32, 0), make_sdesc(ka + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
-        tc_commit(s_full);
-        if (j >= 1 && !do_pv(j - 1)) ok = false;
+          for (int kk = 0; kk < HD / 16; ++kk)
+            tc_mma(tmem + FT_S, make_sdesc(qa + kk * 32, 0), make_sdesc(ka + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+          tc_commit(s_full);
+          if (j == nkv - 1) tc_commit(&q_empty[qbuf]);
+          if (g >= 1 && !do_pv(g - 1, prev_j)) {
+            ok = false;
+            break;
+          }
+          prev_j = j;
+        }
       }
-      if (ok && !do_pv(nkv - 1)) ok = false;
+      if (ok && g >= 1 && !do_pv(g - 1, prev_j)) ok = false;
       if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
       tc_commit(drain);
       if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
@@ -241,112 +304,127 @@ __global__ void __launch_bounds__(192, 2)
     // ---------------------------------------------------- softmax warps
     const int qw = warp & 3;                // TMEM lane quarter
     const int r = qw * 32 + lane;           // query row within the block
-    const int q = qb * BQ + r;              // query position in the sequence
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
-    float m = -INFINITY, l = 0.f;
+    uint32_t g = 0;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!warp_wait(s_full, j & 1u)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // the 128-key row of S in registers (one TMEM wait), buffer released
-      uint32_t v[BKV];
-      tmem_ld64(tl + FT_S, v);
-      tmem_ld64(tl + FT_S + 64, v + 64);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      // causal mask on the block that reaches past the block's first query
-      if (j * BKV + BKV - 1 > qb * BQ) {
-#pragma unroll
-        for (int e = 0; e < BKV; ++e)
-          if (j * BKV + e > q) v[e] = __float_as_uint(-INFINITY);
-      }
-      // row maximum of the raw scores in 8 chains; the positive scale
-      // 1/sqrt(d)*log2(e) is applied to the maximum
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(v[i]);
-#pragma unroll
-      for (int e = 8; e < BKV; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // lazy rescaling: the reference maximum m moves only when some row of
-      // the warp sees a block maximum more than 2^RESCALE_LOG2 above it (and
-      // always for the first block).  O, l and P share the reference, so the
-      // result is exact for any choice of it; P stays <= 2^RESCALE_LOG2.
-      const bool rescale = __any_sync(0xffffffffu, mx * sl2 > m + RESCALE_LOG2);
-      float m_new = m, alpha = 1.f;
-      if (rescale) {
-        m_new = fmaxf(m, mx * sl2);
-        alpha = ex2f(m - m_new);
-      }
-      // p = 2^(s*sl2 - m_new) (one FFMA + ex2), row sum in 8 chains, packed
-      // to bf16 pairs in place
-      float rs8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
-#pragma unroll
-      for (int e = 0; e < BKV; e += 2) {
-        const float p0 = ex2f(fmaf(__uint_as_float(v[e]), sl2, -m_new));
-        const float p1 = ex2f(fmaf(__uint_as_float(v[e + 1]), sl2, -m_new));
-        rs8[e & 7] += p0;
-        rs8[(e + 1) & 7] += p1;
-        v[e >> 1] = pack_bf16x2(p0, p1);
-      }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      l = l * alpha + rs;
-      m = m_new;
-      // O += P_{j-1} V_{j-1} is complete: the P buffer is free and O final up
-      // to block j-1; rescale O in TMEM when the reference moved
-      if (j >= 1) {
-        if (!warp_wait(pv_done, (j - 1) & 1u)) {
+    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+      int qb, bh;
+      item_desc(w, nqb, BH, qb, bh);
+      const int b = bh / H, h = bh % H;
+      const int q = qb * BQ + r;            // query position in the sequence
+      const int nkv = min(qb * BQ + BQ - 1, T - 1) / BKV + 1;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j, ++g) {
+        if (!warp_wait(s_full, g & 1u)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        // the 128-key row of S in registers (one TMEM wait), buffer released
+        uint32_t v[BKV];
+        tmem_ld64(tl + FT_S, v);
+        tmem_ld64(tl + FT_S + 64, v + 64);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // causal mask on the block that reaches past the block's first query
+        if (j * BKV + BKV - 1 > qb * BQ) {
+#pragma unroll
+          for (int e = 0; e < BKV; ++e)
+            if (j * BKV + e > q) v[e] = __float_as_uint(-INFINITY);
+        }
+        // row maximum of the raw scores in 8 chains; the positive scale
+        // 1/sqrt(d)*log2(e) is applied to the maximum
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(v[i]);
+#pragma unroll
+        for (int e = 8; e < BKV; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        // lazy rescaling: the reference maximum m moves only when some row of
+        // the warp sees a block maximum more than 2^RESCALE_LOG2 above it (and
+        // always for the first block).  O, l and P share the reference, so the
+        // result is exact for any choice of it; P stays <= 2^RESCALE_LOG2.
+        const bool rescale = __any_sync(0xffffffffu, mx * sl2 > m + RESCALE_LOG2);
+        float m_new = m, alpha = 1.f;
         if (rescale) {
+          m_new = fmaxf(m, mx * sl2);
+          alpha = ex2f(m - m_new);
+        }
+        // p = 2^(s*sl2 - m_new) (one FFMA + ex2), row sum in 8 chains, packed
+        // to bf16 pairs in place
+        float rs8[8];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t o[32];
-            tmem_ld32(tl + FT_O + half * 32, o);
-            tmem_wait_ld();
+        for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tl + FT_O + half * 32, o);
+        for (int e = 0; e < BKV; e += 2) {
+          // one pair in every EX2_FMA_EVERY goes through the FMA pipe
+          const bool fma_pipe = EX2_FMA_EVERY > 0 && (e / 2) % (EX2_FMA_EVERY > 0 ? EX2_FMA_EVERY : 1) ==
+                                                         (EX2_FMA_EVERY > 0 ? EX2_FMA_EVERY : 1) - 1;
+          const float a0 = fmaf(__uint_as_float(v[e]), sl2, -m_new);
+          const float a1 = fmaf(__uint_as_float(v[e + 1]), sl2, -m_new);
+          const float p0 = fma_pipe ? ex2_fma(a0) : ex2f(a0);
+          const float p1 = fma_pipe ? ex2_fma(a1) : ex2f(a1);
+          rs8[e & 7] += p0;
+          rs8[(e + 1) & 7] += p1;
+          v[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        l = l * alpha + rs;
+        m = m_new;
+        // O += P V of the item's previous block is complete: the P buffer is
+        // free and O final up to it; rescale O in TMEM when the reference
+        // moved.  (For an item's first block the previous item's epilogue
+        // already waited for its last PV.)
+        if (j >= 1) {
+          if (!warp_wait(pv_done, (g - 1) & 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (rescale) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t o[32];
+              tmem_ld32(tl + FT_O + half * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(tl + FT_O + half * 32, o);
+            }
           }
         }
+        tmem_st32(tl + FT_P, v);
+        tmem_st32(tl + FT_P + 32, v + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
       }
-      tmem_st32(tl + FT_P, v);
-      tmem_st32(tl + FT_P + 32, v + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (ok) {
-      if (warp_wait(pv_done, (nkv - 1) & 1u)) {
-        tc_fence_after();
-        uint32_t o[HD];
-        tmem_ld64(tl + FT_O, o);
-        tmem_wait_ld();
-        if (q < T) {
-          const float inv = 1.f / l;
-          bf16* orow = out + ((long)b * T + q) * C + h * HD;
-#pragma unroll
-          for (int i = 0; i < HD; i += 8)
-            *reinterpret_cast<uint4*>(orow + i) = make_uint4(
-                pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv),
-                pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv),
-                pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv),
-                pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv));
-          lse[((long)b * H + h) * T + q] = (m + __log2f(l)) * 0.6931471805599453f;
-        }
-      } else {
+      if (!ok) break;
+      // item epilogue: O / l and the log-sum-exp
+      if (!warp_wait(pv_done, (g - 1) & 1u)) {
         ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t o[HD];
+      tmem_ld64(tl + FT_O, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      if (q < T) {
+        const float inv = 1.f / l;
+        bf16* orow = out + ((long)b * T + q) * C + h * HD;
+#pragma unroll
+        for (int i = 0; i < HD; i += 8)
+          *reinterpret_cast<uint4*>(orow + i) = make_uint4(
+              pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv),
+              pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv),
+              pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv),
+              pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv));
+        lse[((long)b * H + h) * T + q] = (m + __log2f(l)) * 0.6931471805599453f;
       }
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
@@ -356,6 +434,17 @@ __global__ void __launch_bounds__(192, 2)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(F_TMEM_COLS) : "memory");
   }
+}
+
+static int num_sms_attn() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
 }
 
 static inline cudaError_t forward(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, cudaStream_t st) {
@@ -370,8 +459,9 @@ static inline cudaError_t forward(const bf16* qkv, bf16* out, float* lse, int B,
   const int C = H * HD;
   if (make_tmap(&tm, qkv, 3L * C, (long)B * T, 3L * C, 64, BKV) != 0) return cudaErrorInvalidValue;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
-  dim3 grid((T + BQ - 1) / BQ, B * H);
-  fwd_kernel<<<grid, 192, F_SMEM, st>>>(tm, out, lse, T, H, sl2);
+  const int items = ((T + BQ - 1) / BQ) * B * H;
+  const int grid = items < 2 * num_sms_attn() ? items : 2 * num_sms_attn();
+  fwd_kernel<<<grid, 192, F_SMEM, st>>>(tm, out, lse, T, H, B * H, sl2);
   return cudaGetLastError();
 }
 

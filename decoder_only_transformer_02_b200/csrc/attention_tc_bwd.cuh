@@ -3,37 +3,46 @@
 // With P = exp(S/sqrt(d) - lse) and D_q = sum_d dO_q . O_q:
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dK = dS^T Q / sqrt(d),
 //   dQ = dS K / sqrt(d).
-// Two deterministic kernels (no atomics), each with one CTA per SM and
-// 128 x 128 score tiles:
-//  dq_kernel (runs first): one CTA owns 128 queries of one (batch, head) and
+// Two deterministic kernels (no atomics), each persistent with one CTA per SM
+// and 128 x 128 score tiles.  A CTA takes work items in a fixed order, longest
+// first, and its pipeline runs across item boundaries (the next item's tiles
+// load and its first MMAs run while the current item's results are written).
+//  dq_kernel (runs first): an item is 128 queries of one (batch, head); it
 //     walks the 128-key blocks up to its last query:
 //       S = Q K_j^T, dP = dO V_j^T        (M=128 queries, N=128 keys, K=64)
-//       dS = P * (dP - D)                  (eight compute warps, bf16 into TMEM)
+//       dS = P * (dP - D)                  (sixteen compute warps, bf16 into TMEM)
 //       dQ += dS K_j                       (A = dS read from TMEM, K=128 keys)
 //     It also forms D for its queries (from the dO tile in shared memory and
-//     the rows of O) and writes lse*log2(e) and D per 128-query block into a
-//     padded fp32 array (+inf / 0 past T) that dkdv_kernel streams by bulk copy.
-//  dkdv_kernel: one CTA owns 128 keys and walks the 128-query blocks that
-//     reach them:
+//     the rows of O; one warp per lane quarter, shared with the other three
+//     through shared memory) and writes lse*log2(e) and D per 128-query block
+//     into a padded fp32 array (+inf / 0 past T) that dkdv_kernel streams by
+//     bulk copy.
+//  dkdv_kernel: an item is 128 keys of one (batch, head); it walks the
+//     128-query blocks that reach them:
 //       S^T = K Q_i^T, dP^T = V dO_i^T     (M=128 keys, N=128 queries, K=64)
 //       P^T, dS^T                          (bf16 into TMEM)
 //       dV += P^T dO_i, dK += dS^T Q_i     (A from TMEM, K=128 queries)
 // The score tiles never touch shared memory: S and dP are read from TMEM into
 // registers, and P / dS go back into TMEM as the A operand of the next MMAs.
 // Warp 0 streams the operand tiles through a 4-stage TMA ring, warp 1 issues
-// the MMAs (one thread), warps 2..9 do the element-wise math: warps w and w+4
-// share TMEM lane quarter w%4 (one row each) and take the two 64-column halves
-// of the tile.  While the warps work on tile j, the tensor cores already run
-// S_{j+1} and dP_{j+1} (and the accumulating MMAs of tile j-1).  Every wait is
-// bounded; the waits that drain a CTA's own copies and MMAs before it exits
-// have their own fixed limit.
+// the MMAs (one thread), warps 2..17 do the element-wise math: warps w, w+4,
+// w+8 and w+12 share TMEM lane quarter w%4 (one row each) and take the four
+// 32-column quarters of the tile, so every SM sub-partition has four warps to
+// hide the TMEM and shared-memory latencies with.  While the warps work on tile j, the tensor cores already run
+// S_{j+1} and dP_{j+1} (and the accumulating MMAs of tile j-1).  Both kernels
+// can also write per-(128-row block, lane quarter) column sums of what they
+// store (the qkv bias gradient).  Every wait is bounded; the waits that drain
+// a CTA's own copies and MMAs before it exits have their own fixed limit.
 #pragma once
 #include "attention.cuh"
 #include "attention_tc.cuh"
 
 namespace tcfa {
 
-constexpr int BW_THREADS = 320;               // producer, MMA issuer, 8 compute warps
+constexpr int BW_CWARPS = 16;                 // compute warps: four per TMEM lane quarter
+constexpr int BW_THREADS = 64 + 32 * BW_CWARPS; // producer, MMA issuer, compute warps
+constexpr int BW_CW = 128 / (BW_CWARPS / 4);    // score-tile columns per compute warp (32)
+constexpr int BW_EW = 64 / (BW_CWARPS / 4);     // accumulator columns per compute warp (16)
 constexpr int BW_STAGES = 4;                  // operand ring depth
 constexpr int BT = 128;                       // rows of a score tile (queries or keys)
 constexpr int LD_FLOATS = 2 * BT;             // per 128-query block: lse*log2(e)[128], D[128]
@@ -50,56 +59,114 @@ __device__ __forceinline__ void store_row32(bf16* dst, const uint32_t (&a)[32], 
         pack_bf16x2(__uint_as_float(a[e + 6]) * scale, __uint_as_float(a[e + 7]) * scale));
 }
 
+__device__ __forceinline__ void store_row16(bf16* dst, const uint32_t (&a)[16], float scale) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 8)
+    *reinterpret_cast<uint4*>(dst + e) = make_uint4(
+        pack_bf16x2(__uint_as_float(a[e]) * scale, __uint_as_float(a[e + 1]) * scale),
+        pack_bf16x2(__uint_as_float(a[e + 2]) * scale, __uint_as_float(a[e + 3]) * scale),
+        pack_bf16x2(__uint_as_float(a[e + 4]) * scale, __uint_as_float(a[e + 5]) * scale),
+        pack_bf16x2(__uint_as_float(a[e + 6]) * scale, __uint_as_float(a[e + 7]) * scale));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+// Transposing warp reduction of 16 columns: lane L holds v[0..15] (one row);
+// returns to lanes L and L+16 the sum over the 32 lanes of column L (L < 16),
+// in a fixed order.
+__device__ __forceinline__ float warp_colsum16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = up ? v[i] : v[i + w];
+      const float keep = up ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+static_assert(BW_CW == 32 && BW_EW == 16, "the compute-warp code below handles 32 score and 16 output columns");
+
+// wait (bounded) until every issued phase of a ring of n barriers has
+// completed: the drain of a CTA's own in-flight copies before it exits
+__device__ __forceinline__ void drain_ring(uint64_t* bars, int n, uint32_t issued) {
+  for (int s = 0; s < n; ++s) {
+    if ((uint32_t)s < issued) {
+      const uint32_t last = issued - 1 - ((issued - 1 - s) % n);
+      if (!mbar_wait_drain(&bars[s], (last / n) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  }
+}
+
 // ----------------------------------------------------------------- dQ
-// Shared memory: Q 128x64, dO 128x64 (16 KB each, 128-byte swizzled K-major
-// rows of 64 bf16), then the ring of K_j, V_j tiles (32 KB per stage).
-constexpr int DQ_Q_OFF = 0;
-constexpr int DQ_DO_OFF = TILE;
-constexpr int DQ_RING_OFF = 2 * TILE;  // stage s: K at +2s*TILE, V at +(2s+1)*TILE
-constexpr int DQ_BAR_OFF = DQ_RING_OFF + 2 * BW_STAGES * TILE;
-constexpr int DQ_RED_OFF = DQ_BAR_OFF + 256;
-constexpr int DQ_SMEM = DQ_RED_OFF + 2 * 4 * 32 * 4 + 1024;
-// TMEM columns: S [0,128), dP [128,256), dQ [256,320), dS (bf16 pairs) [320,384)
-constexpr uint32_t DQ_T_S = 0, DQ_T_DP = 128, DQ_T_DQ = 256, DQ_T_DS = 320;
+// Shared memory: two buffers of (Q, dO) 128x64 tiles (16 KB each, 128-byte
+// swizzled K-major rows of 64 bf16), then the ring of K_j, V_j tiles.
+constexpr int DQ_QD_OFF = 0;                               // buffer b: Q at +2b*TILE, dO at +(2b+1)*TILE
+constexpr int DQ_RING_OFF = 4 * TILE;                      // stage s: K at +2s*TILE, V at +(2s+1)*TILE
+constexpr int DQ_D_OFF = DQ_RING_OFF + 2 * BW_STAGES * TILE;  // per item parity: lse*log2(e)[128], D[128]
+constexpr int DQ_BAR_OFF = DQ_D_OFF + 2 * 2 * BT * 4;
+constexpr int DQ_SMEM = DQ_BAR_OFF + 256 + 1024;
+// TMEM columns: S [0,128), dP [128,256), dQ of item parity 0 / 1 [256,320) /
+// [320,384), dS (bf16 pairs) [384,448)
+constexpr uint32_t DQ_T_S = 0, DQ_T_DP = 128, DQ_T_DQ = 256, DQ_T_DS = 384;
 
 __global__ void __launch_bounds__(BW_THREADS, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
               const bf16* __restrict__ out, const float* __restrict__ lse, float* __restrict__ ld_out,
-              bf16* __restrict__ dqkv, float* __restrict__ colsum, int T, int H, float scale, float sl2) {
+              bf16* __restrict__ dqkv, float* __restrict__ colsum, int T, int H, int BH, float scale, float sl2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_BAR_OFF);
-  uint64_t* q_full = bars;                   // Q and dO tiles landed
-  uint64_t* kv_full = bars + 1;              // BW_STAGES
+  uint64_t* q_full = bars;                   // 2: Q and dO tiles landed
+  uint64_t* q_empty = bars + 2;              // 2, count 5: last S/dP MMA done and D formed
+  uint64_t* kv_full = bars + 4;              // BW_STAGES
   uint64_t* kv_empty = kv_full + BW_STAGES;  // BW_STAGES
-  uint64_t* s_full = kv_empty + BW_STAGES;   // S_j and dP_j in TMEM
-  uint64_t* s_free = s_full + 1;             // count 8: S_j and dP_j are in registers
-  uint64_t* ds_full = s_free + 1;            // count 8: dS_j in TMEM
-  uint64_t* ds_free = ds_full + 1;           // dQ += dS_j K_j has read dS_j
-  uint64_t* acc_done = ds_free + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
-  float* red = reinterpret_cast<float*>(smem + DQ_RED_OFF);  // [2 halves][4 quarters][32]
+  uint64_t* s_full = kv_empty + BW_STAGES;   // S and dP in TMEM
+  uint64_t* s_free = s_full + 1;             // count BW_CWARPS: S and dP are in registers
+  uint64_t* ds_full = s_free + 1;            // count BW_CWARPS: dS in TMEM
+  uint64_t* ds_free = ds_full + 1;           // dQ += dS K has read dS
+  uint64_t* acc_full = ds_free + 1;          // 2: the item's dQ is complete
+  uint64_t* acc_empty = acc_full + 2;        // 2, count 16: the item's dQ is in registers
+  uint64_t* d_ready = acc_empty + 2;         // count 4: the item's lse*log2(e) and D are in shared memory
+  uint64_t* drain = d_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqb = gridDim.x;
-  const int qb = nqb - 1 - blockIdx.x;  // most key blocks first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int nqb = (T + BT - 1) / BT;
+  const int nitems = nqb * BH;
   const int C = H * HD;
-  const int row0 = b * T;
-  const int qlast = min(qb * BT + BT - 1, T - 1);
-  const int nblk = qlast / BT + 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1 + BW_CWARPS / 4);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], BW_CWARPS);
+    }
     for (int s = 0; s < BW_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
-    mbar_init(ds_full, 8);
+    mbar_init(s_free, BW_CWARPS);
+    mbar_init(ds_full, BW_CWARPS);
     mbar_init(ds_free, 1);
-    mbar_init(acc_done, 1);
+    mbar_init(d_ready, BW_CWARPS / 4);
+    mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -118,191 +185,244 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       // -------------------------------------------------------- producer
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_do)) : "memory");
-      mbar_expect_tx(q_full, 2 * TILE);
-      tma_load_2d(smem_u32(smem + DQ_Q_OFF), &tm_qkv, h * HD, row0 + qb * BT, q_full);
-      tma_load_2d(smem_u32(smem + DQ_DO_OFF), &tm_do, h * HD, row0 + qb * BT, q_full);
-      uint32_t issued = 0;
-      for (int j = 0; j < nblk; ++j, ++issued) {
-        const int s = j % BW_STAGES;
-        if (!mbar_wait(&kv_empty[s], ((j / BW_STAGES) & 1u) ^ 1u)) {
-          set_device_err(DERR_WAIT_TIMEOUT);
+      uint32_t g = 0, t = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int qb, bh;
+        item_desc(w, nqb, BH, qb, bh);
+        const int b = bh / H, h = bh % H, row0 = b * T;
+        const int nblk = min(qb * BT + BT - 1, T - 1) / BT + 1;
+        const uint32_t qbuf = t & 1u;
+        if (!mbar_wait(&q_empty[qbuf], ((t >> 1) & 1u) ^ 1u)) {
+          ok = false;
           break;
         }
-        mbar_expect_tx(&kv_full[s], 2 * TILE);
-        const uint32_t dst = smem_u32(smem + DQ_RING_OFF + 2 * s * TILE);
-        tma_load_2d(dst, &tm_qkv, C + h * HD, row0 + j * BT, &kv_full[s]);
-        tma_load_2d(dst + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BT, &kv_full[s]);
-      }
-      // drain: every issued load has landed before the CTA exits
-      for (int s = 0; s < BW_STAGES; ++s) {
-        if ((uint32_t)s < issued) {
-          const uint32_t last = issued - 1 - ((issued - 1 - s) % BW_STAGES);
-          if (!mbar_wait_drain(&kv_full[s], (last / BW_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        mbar_expect_tx(&q_full[qbuf], 2 * TILE);
+        const uint32_t qd = smem_u32(smem + DQ_QD_OFF + 2 * qbuf * TILE);
+        tma_load_2d(qd, &tm_qkv, h * HD, row0 + qb * BT, &q_full[qbuf]);
+        tma_load_2d(qd + TILE, &tm_do, h * HD, row0 + qb * BT, &q_full[qbuf]);
+        for (int j = 0; j < nblk; ++j, ++g) {
+          const int s = g % BW_STAGES;
+          if (!mbar_wait(&kv_empty[s], ((g / BW_STAGES) & 1u) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&kv_full[s], 2 * TILE);
+          const uint32_t dst = smem_u32(smem + DQ_RING_OFF + 2 * s * TILE);
+          tma_load_2d(dst, &tm_qkv, C + h * HD, row0 + j * BT, &kv_full[s]);
+          tma_load_2d(dst + TILE, &tm_qkv, 2 * C + h * HD, row0 + j * BT, &kv_full[s]);
         }
       }
-      if (!mbar_wait_drain(q_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      drain_ring(kv_full, BW_STAGES, g);
+      drain_ring(q_full, 2, t);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer
       constexpr uint32_t id_s = att_idesc(BT, 0);   // S, dP: N = 128 keys, K = 64 (d)
       constexpr uint32_t id_dq = att_idesc(HD, 1);  // dQ: N = 64 (d), K = 128 keys, K_j MN-major
-      bool ok = mbar_wait(q_full, 0);
-      const uint32_t qa = smem_u32(smem + DQ_Q_OFF), doa = smem_u32(smem + DQ_DO_OFF);
-      auto dq_step = [&](int i) -> bool {
-        if (!mbar_wait(ds_full, i & 1u)) return false;
+      uint32_t g = 0, t = 0;
+      int pj = 0, plast = 0;   // step g-1: block index within its item, last block of it?
+      uint32_t pt = 0;         // step g-1: item counter
+      bool ok = true;
+      auto dq_step = [&](uint32_t gp, int jp, uint32_t tp, int last) -> bool {
+        const uint32_t ab = tp & 1u;
+        if (jp == 0 && !mbar_wait(&acc_empty[ab], ((tp >> 1) & 1u) ^ 1u)) return false;
+        if (!mbar_wait(ds_full, gp & 1u)) return false;
         tc_fence_after();
-        const uint32_t ka = smem_u32(smem + DQ_RING_OFF + 2 * (i % BW_STAGES) * TILE);
+        const uint32_t ka = smem_u32(smem + DQ_RING_OFF + 2 * (gp % BW_STAGES) * TILE);
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          tc_mma_ts(tmem + DQ_T_DQ, tmem + DQ_T_DS + kk * 8, make_sdesc(ka + kk * 2048, 1), id_dq,
-                    (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&kv_empty[i % BW_STAGES]);
+          tc_mma_ts(tmem + DQ_T_DQ + ab * HD, tmem + DQ_T_DS + kk * 8, make_sdesc(ka + kk * 2048, 1), id_dq,
+                    (jp > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&kv_empty[gp % BW_STAGES]);
         tc_commit(ds_free);
+        if (last) tc_commit(&acc_full[ab]);
         return true;
       };
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int s = j % BW_STAGES;
-        if (!mbar_wait(&kv_full[s], (j / BW_STAGES) & 1u)) {
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int qb, bh;
+        item_desc(w, nqb, BH, qb, bh);
+        const int nblk = min(qb * BT + BT - 1, T - 1) / BT + 1;
+        const uint32_t qbuf = t & 1u;
+        if (!mbar_wait(&q_full[qbuf], (t >> 1) & 1u)) {
           ok = false;
           break;
         }
-        if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t ka = smem_u32(smem + DQ_RING_OFF + 2 * s * TILE);
-        const uint32_t va = ka + TILE;
+        const uint32_t qa = smem_u32(smem + DQ_QD_OFF + 2 * qbuf * TILE), doa = qa + TILE;
+        for (int j = 0; j < nblk; ++j, ++g) {
+          const int s = g % BW_STAGES;
+          if (!mbar_wait(&kv_full[s], (g / BW_STAGES) & 1u) || (g >= 1 && !mbar_wait(s_free, (g - 1) & 1u))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(smem + DQ_RING_OFF + 2 * s * TILE);
+          const uint32_t va = ka + TILE;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          tc_mma(tmem + DQ_T_S, make_sdesc(qa + kk * 32, 0), make_sdesc(ka + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
-          tc_mma(tmem + DQ_T_DP, make_sdesc(doa + kk * 32, 0), make_sdesc(va + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            tc_mma(tmem + DQ_T_S, make_sdesc(qa + kk * 32, 0), make_sdesc(ka + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+            tc_mma(tmem + DQ_T_DP, make_sdesc(doa + kk * 32, 0), make_sdesc(va + kk * 32, 0), id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full);
+          if (j == nblk - 1) tc_commit(&q_empty[qbuf]);
+          if (g >= 1 && !dq_step(g - 1, pj, pt, plast)) {
+            ok = false;
+            break;
+          }
+          pj = j;
+          pt = t;
+          plast = j == nblk - 1;
         }
-        tc_commit(s_full);
-        if (j >= 1 && !dq_step(j - 1)) ok = false;
       }
-      if (ok && !dq_step(nblk - 1)) ok = false;
+      if (ok && g >= 1 && !dq_step(g - 1, pj, pt, plast)) ok = false;
       if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
-      tc_commit(acc_done);
-      if (!mbar_wait_drain(acc_done, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_commit(drain);
+      if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
     }
   } else {
     // ---------------------------------------------------- compute warps
     const int qw = warp & 3;             // TMEM lane quarter
-    const int hf = (warp - 2) >> 2;      // which 64 keys of the 128-key tile
+    const int cq = (warp - 2) >> 2;      // which 32 keys of the 128-key tile (and 16 dQ columns)
     const int r = qw * 32 + lane;        // query row within the block
-    const int q = qb * BT + r;           // query position
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
-    const float l2 = q < T ? lse[(long)bh * T + q] * 1.4426950408889634f : INFINITY;
-    bool ok = warp_wait(q_full, 0);
-    // D_q = sum_d dO[q,d] O[q,d] (the row of O from global memory, dO from the
-    // tile in shared memory)
-    float dq_ = 0.f;
-    if (ok && q < T) {
-      const bf16* orow = out + ((long)row0 + q) * C + h * HD;
-      const uint8_t* dorow = smem + DQ_DO_OFF;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float* Dsm = reinterpret_cast<float*>(smem + DQ_D_OFF);  // [item parity][lse2 128, D 128]
+    uint32_t g = 0, t = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      int qb, bh;
+      item_desc(w, nqb, BH, qb, bh);
+      const int b = bh / H, h = bh % H, row0 = b * T;
+      const int q = qb * BT + r;          // query position
+      const int nblk = min(qb * BT + BT - 1, T - 1) / BT + 1;
+      const uint32_t qbuf = t & 1u;
+      float* dsm = Dsm + (t & 1u) * 2 * BT;
+      if (cq == 0) {
+        // D_q = sum_d dO[q,d] O[q,d] (the row of O from global memory, dO
+        // from the tile in shared memory) and lse*log2(e), for the item's
+        // four warps of this lane quarter and for dkdv_kernel
+        const float l2 = q < T ? lse[(long)bh * T + q] * 1.4426950408889634f : INFINITY;
+        if (!warp_wait(&q_full[qbuf], (t >> 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        float dq_ = 0.f;
+        if (q < T) {
+          const bf16* orow = out + ((long)row0 + q) * C + h * HD;
+          const uint8_t* dorow = smem + DQ_QD_OFF + (2 * qbuf + 1) * TILE;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < HD / 8; ++c) {
-        const uint4 ov = *reinterpret_cast<const uint4*>(orow + 8 * c);
-        const uint4 dv = *reinterpret_cast<const uint4*>(dorow + sw128(r, c));
-        const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w}, d4[4] = {dv.x, dv.y, dv.z, dv.w};
+          for (int c = 0; c < HD / 8; ++c) {
+            const uint4 ov = *reinterpret_cast<const uint4*>(orow + 8 * c);
+            const uint4 dv = *reinterpret_cast<const uint4*>(dorow + sw128(r, c));
+            const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w}, d4[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 of = unpack_bf16x2(o4[e]), df = unpack_bf16x2(d4[e]);
-          acc[e] = fmaf(of.x, df.x, fmaf(of.y, df.y, acc[e]));
+            for (int e = 0; e < 4; ++e) {
+              const float2 of = unpack_bf16x2(o4[e]), df = unpack_bf16x2(d4[e]);
+              acc[e] = fmaf(of.x, df.x, fmaf(of.y, df.y, acc[e]));
+            }
+          }
+          dq_ = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+        dsm[r] = l2;
+        dsm[BT + r] = dq_;
+        float* ldb = ld_out + ((long)bh * nqb + qb) * LD_FLOATS;
+        ldb[r] = l2;
+        ldb[BT + r] = dq_;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&q_empty[qbuf]);  // this warp is done with the dO tile
+          mbar_arrive(d_ready);
         }
       }
-      dq_ = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    }
-    if (ok && hf == 0) {
-      float* ldb = ld_out + ((long)bh * nqb + qb) * LD_FLOATS;
-      ldb[r] = l2;
-      ldb[BT + r] = dq_;
-    }
-    for (int j = 0; ok && j < nblk; ++j) {
-      if (!warp_wait(s_full, j & 1u)) {
+      if (!warp_wait(d_ready, t & 1u)) {
+        ok = false;
+        break;
+      }
+      const float l2 = dsm[r], dq_ = dsm[BT + r];
+      for (int j = 0; j < nblk; ++j, ++g) {
+        if (!warp_wait(s_full, g & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tl + DQ_T_S + cq * 32, sv);
+        tmem_ld32(tl + DQ_T_DP + cq * 32, dv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        const int k0 = j * BT + cq * 32;      // first key of this warp's columns
+        const bool diag = k0 + 31 > qb * BT;  // some key of the columns follows some query of the block
+        // dS = P * (dP - D), packed to bf16 pairs in place
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const bool fma_pipe = EX2_FMA_EVERY > 0 && (c / 2) % (EX2_FMA_EVERY > 0 ? EX2_FMA_EVERY : 1) ==
+                                                         (EX2_FMA_EVERY > 0 ? EX2_FMA_EVERY : 1) - 1;
+          const float a0 = fmaf(__uint_as_float(sv[c]), sl2, -l2), a1 = fmaf(__uint_as_float(sv[c + 1]), sl2, -l2);
+          float p0 = fma_pipe ? ex2_fma(a0) : ex2f(a0);
+          float p1 = fma_pipe ? ex2_fma(a1) : ex2f(a1);
+          if (diag) {
+            if (k0 + c > q) p0 = 0.f;
+            if (k0 + c + 1 > q) p1 = 0.f;
+          }
+          sv[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - dq_), p1 * (__uint_as_float(dv[c + 1]) - dq_));
+        }
+        // the previous step's dQ MMA has read the dS buffer
+        if (g >= 1 && !warp_wait(ds_free, (g - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tl + DQ_T_DS + cq * 16, sv);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
+      }
+      if (!ok) break;
+      // item epilogue: dQ (scaled) and its column sums
+      const uint32_t ab = t & 1u;
+      if (!warp_wait(&acc_full[ab], (t >> 1) & 1u)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[64], dv[64];
-      tmem_ld64(tl + DQ_T_S + hf * 64, sv);
-      tmem_ld64(tl + DQ_T_DP + hf * 64, dv);
+      uint32_t a[16];
+      tmem_ld16(tl + DQ_T_DQ + ab * HD + cq * 16, a);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      const int k0 = j * BT + hf * 64;      // first key of this warp's columns
-      const bool diag = k0 + 63 > qb * BT;  // some key of the columns follows some query of the block
-      // dS = P * (dP - D), packed to bf16 pairs in place
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      float cs[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float p0 = ex2f(fmaf(__uint_as_float(sv[c]), sl2, -l2));
-        float p1 = ex2f(fmaf(__uint_as_float(sv[c + 1]), sl2, -l2));
-        if (diag) {
-          if (k0 + c > q) p0 = 0.f;
-          if (k0 + c + 1 > q) p1 = 0.f;
-        }
-        sv[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - dq_), p1 * (__uint_as_float(dv[c + 1]) - dq_));
+      for (int i = 0; i < 16; ++i) cs[i] = q < T ? __uint_as_float(a[i]) * scale : 0.f;
+      if (q < T) store_row16(dqkv + ((long)row0 + q) * (3L * C) + h * HD + cq * 16, a, scale);
+      if (colsum) {
+        const float tot = warp_colsum16(cs, lane);
+        if (lane < 16) colsum[(((long)b * nqb + qb) * 4 + qw) * (3L * C) + h * HD + cq * 16 + lane] = tot;
       }
-      // dQ += dS_{j-1} K_{j-1} has read the dS buffer
-      if (j >= 1 && !warp_wait(ds_free, (j - 1) & 1u)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st32(tl + DQ_T_DS + hf * 32, sv);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    float cs[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) cs[i] = 0.f;
-    if (ok && warp_wait(acc_done, 0)) {
-      tc_fence_after();
-      uint32_t a[32];
-      tmem_ld32(tl + DQ_T_DQ + hf * 32, a);
-      tmem_wait_ld();
-      if (q < T) {
-        store_row32(dqkv + ((long)row0 + q) * (3L * C) + h * HD + hf * 32, a, scale);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) cs[i] = __uint_as_float(a[i]) * scale;
-      }
-    } else {
-      ok = false;
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
-    if (colsum) red[(hf * 4 + qw) * 32 + lane] = warp_colsum32(cs, lane);
   }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BW_TMEM_COLS) : "memory");
   }
-  // column sums of dQ over the block's rows (the query bias gradient), as
-  // one partial row per 128-row block, quarters added in a fixed order
-  if (colsum && warp >= 2 && warp < 4) {
-    const int hf = warp - 2;
-    const float t = ((red[(hf * 4) * 32 + lane] + red[(hf * 4 + 1) * 32 + lane]) + red[(hf * 4 + 2) * 32 + lane]) +
-                    red[(hf * 4 + 3) * 32 + lane];
-    colsum[((long)b * nqb + qb) * (3L * C) + h * HD + hf * 32 + lane] = t;
-  }
 }
 
 // ------------------------------------------------------------ dK, dV
-// Shared memory: K, V 128x64 (16 KB each), then the ring of Q_i, dO_i tiles and
-// the block's lse*log2(e) / D rows (33 KB per stage).
-constexpr int DKV_K_OFF = 0;
-constexpr int DKV_V_OFF = TILE;
+// Shared memory: two buffers of (K, V) 128x64 tiles, then the ring of Q_i,
+// dO_i tiles and the block's lse*log2(e) / D rows (33 KB per stage).
+constexpr int DKV_KV_OFF = 0;                              // buffer b: K at +2b*TILE, V at +(2b+1)*TILE
 constexpr int DKV_STAGE_BYTES = 2 * TILE + LD_FLOATS * 4;
-constexpr int DKV_RING_OFF = 2 * TILE;  // stage s: Q, dO, lse2/D
+constexpr int DKV_RING_OFF = 4 * TILE;                     // stage s: Q, dO, lse2/D
 constexpr int DKV_BAR_OFF = DKV_RING_OFF + BW_STAGES * DKV_STAGE_BYTES;
-constexpr int DKV_RED_OFF = DKV_BAR_OFF + 256;
-constexpr int DKV_SMEM = DKV_RED_OFF + 2 * 2 * 4 * 32 * 4 + 1024;
+constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
 // P^T (bf16 pairs) [384,448), dS^T (bf16 pairs) [448,512)
 constexpr uint32_t DKV_T_S = 0, DKV_T_DP = 128, DKV_T_DV = 256, DKV_T_DK = 320, DKV_T_P = 384, DKV_T_DS = 448;
@@ -311,40 +431,42 @@ static_assert(DKV_STAGE_BYTES % 1024 == 0, "ring stages keep the 1024-byte swizz
 __global__ void __launch_bounds__(BW_THREADS, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
                 const float* __restrict__ ld_in, bf16* __restrict__ dqkv, float* __restrict__ colsum, int T, int H,
-                float scale, float sl2) {
+                int BH, float scale, float sl2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
-  uint64_t* kv_full = bars;                  // K and V tiles
-  uint64_t* qd_full = bars + 1;              // BW_STAGES
+  uint64_t* kv_full = bars;                  // 2: K and V tiles
+  uint64_t* kv_empty = bars + 2;             // 2: the item's last S^T / dP^T MMA has read them
+  uint64_t* qd_full = bars + 4;              // BW_STAGES
   uint64_t* qd_empty = qd_full + BW_STAGES;  // BW_STAGES
   uint64_t* s_full = qd_empty + BW_STAGES;   // S^T and dP^T in TMEM
-  uint64_t* s_free = s_full + 1;             // count 8
-  uint64_t* p_full = s_free + 1;             // count 8: P^T and dS^T in TMEM
+  uint64_t* s_free = s_full + 1;             // count BW_CWARPS
+  uint64_t* p_full = s_free + 1;             // count BW_CWARPS: P^T and dS^T in TMEM
   uint64_t* p_free = p_full + 1;             // the dV / dK MMAs have read them
-  uint64_t* acc_done = p_free + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
-  float* red = reinterpret_cast<float*>(smem + DKV_RED_OFF);  // [dK, dV][2 halves][4 quarters][32]
+  uint64_t* acc_done = p_free + 1;           // the item's dV / dK are complete
+  uint64_t* drain = acc_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqb = gridDim.x;
-  const int kb = blockIdx.x;  // key block; small kb = most query blocks, launched first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int nqb = (T + BT - 1) / BT;
+  const int nitems = nqb * BH;
   const int C = H * HD;
-  const int row0 = b * T;
-  const int nblk = nqb - kb;  // query blocks kb .. nqb-1
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
     for (int s = 0; s < BW_STAGES; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
-    mbar_init(p_full, 8);
+    mbar_init(s_free, BW_CWARPS);
+    mbar_init(p_full, BW_CWARPS);
     mbar_init(p_free, 1);
     mbar_init(acc_done, 1);
+    mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -358,188 +480,227 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // items in ascending key block: key block 0 meets the most query blocks
+  auto item = [&](int w, int& kb, int& bh) {
+    kb = w / BH;
+    bh = w % BH;
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       // -------------------------------------------------------- producer
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_do)) : "memory");
-      mbar_expect_tx(kv_full, 2 * TILE);
-      tma_load_2d(smem_u32(smem + DKV_K_OFF), &tm_qkv, C + h * HD, row0 + kb * BT, kv_full);
-      tma_load_2d(smem_u32(smem + DKV_V_OFF), &tm_qkv, 2 * C + h * HD, row0 + kb * BT, kv_full);
-      uint32_t issued = 0;
-      for (int n = 0; n < nblk; ++n, ++issued) {
-        const int i = kb + n, s = n % BW_STAGES;
-        if (!mbar_wait(&qd_empty[s], ((n / BW_STAGES) & 1u) ^ 1u)) {
-          set_device_err(DERR_WAIT_TIMEOUT);
+      uint32_t g = 0, t = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int kb, bh;
+        item(w, kb, bh);
+        const int b = bh / H, h = bh % H, row0 = b * T;
+        const int nblk = nqb - kb;  // query blocks kb .. nqb-1
+        const uint32_t kvb = t & 1u;
+        if (!mbar_wait(&kv_empty[kvb], ((t >> 1) & 1u) ^ 1u)) {
+          ok = false;
           break;
         }
-        mbar_expect_tx(&qd_full[s], DKV_STAGE_BYTES);
-        const uint32_t dst = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
-        tma_load_2d(dst, &tm_qkv, h * HD, row0 + i * BT, &qd_full[s]);
-        tma_load_2d(dst + TILE, &tm_do, h * HD, row0 + i * BT, &qd_full[s]);
-        bulk_load(dst + 2 * TILE, ld_in + ((long)bh * nqb + i) * LD_FLOATS, LD_FLOATS * 4, &qd_full[s]);
-      }
-      // drain: every issued load has landed before the CTA exits
-      for (int s = 0; s < BW_STAGES; ++s) {
-        if ((uint32_t)s < issued) {
-          const uint32_t last = issued - 1 - ((issued - 1 - s) % BW_STAGES);
-          if (!mbar_wait_drain(&qd_full[s], (last / BW_STAGES) & 1u)) set_device_err(DERR_WAIT_TIMEOUT);
+        mbar_expect_tx(&kv_full[kvb], 2 * TILE);
+        const uint32_t kd = smem_u32(smem + DKV_KV_OFF + 2 * kvb * TILE);
+        tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + kb * BT, &kv_full[kvb]);
+        tma_load_2d(kd + TILE, &tm_qkv, 2 * C + h * HD, row0 + kb * BT, &kv_full[kvb]);
+        for (int n = 0; n < nblk; ++n, ++g) {
+          const int i = kb + n, s = g % BW_STAGES;
+          if (!mbar_wait(&qd_empty[s], ((g / BW_STAGES) & 1u) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&qd_full[s], DKV_STAGE_BYTES);
+          const uint32_t dst = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
+          tma_load_2d(dst, &tm_qkv, h * HD, row0 + i * BT, &qd_full[s]);
+          tma_load_2d(dst + TILE, &tm_do, h * HD, row0 + i * BT, &qd_full[s]);
+          bulk_load(dst + 2 * TILE, ld_in + ((long)bh * nqb + i) * LD_FLOATS, LD_FLOATS * 4, &qd_full[s]);
         }
       }
-      if (!mbar_wait_drain(kv_full, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      drain_ring(qd_full, BW_STAGES, g);
+      drain_ring(kv_full, 2, t);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer
       constexpr uint32_t id_s = att_idesc(BT, 0);    // S^T, dP^T: N = 128 queries, K = 64 (d)
       constexpr uint32_t id_acc = att_idesc(HD, 1);  // dV, dK: N = 64 (d), K = 128 queries, B MN-major
-      bool ok = mbar_wait(kv_full, 0);
-      const uint32_t ka = smem_u32(smem + DKV_K_OFF), va = smem_u32(smem + DKV_V_OFF);
-      auto acc_step = [&](int n) -> bool {
-        if (!mbar_wait(p_full, n & 1u)) return false;
+      uint32_t g = 0, t = 0;
+      int pn = 0, plast = 0;  // step g-1: block index within its item, last block of it?
+      bool ok = true;
+      auto acc_step = [&](uint32_t gp, int np, int last) -> bool {
+        if (!mbar_wait(p_full, gp & 1u)) return false;
         tc_fence_after();
-        const int s = n % BW_STAGES;
+        const int s = gp % BW_STAGES;
         const uint32_t qa = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
         const uint32_t doa = qa + TILE;
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t acc = (np > 0 || kk > 0) ? 1u : 0u;
           tc_mma_ts(tmem + DKV_T_DV, tmem + DKV_T_P + kk * 8, make_sdesc(doa + kk * 2048, 1), id_acc, acc);
           tc_mma_ts(tmem + DKV_T_DK, tmem + DKV_T_DS + kk * 8, make_sdesc(qa + kk * 2048, 1), id_acc, acc);
         }
         tc_commit(&qd_empty[s]);
         tc_commit(p_free);
+        if (last) tc_commit(acc_done);
         return true;
       };
-      for (int n = 0; ok && n < nblk; ++n) {
-        const int s = n % BW_STAGES;
-        if (!mbar_wait(&qd_full[s], (n / BW_STAGES) & 1u)) {
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int kb, bh;
+        item(w, kb, bh);
+        const int nblk = nqb - kb;
+        const uint32_t kvb = t & 1u;
+        if (!mbar_wait(&kv_full[kvb], (t >> 1) & 1u)) {
           ok = false;
           break;
         }
-        if (n >= 1 && !mbar_wait(s_free, (n - 1) & 1u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t qa = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
-        const uint32_t doa = qa + TILE;
+        const uint32_t ka = smem_u32(smem + DKV_KV_OFF + 2 * kvb * TILE), va = ka + TILE;
+        for (int n = 0; n < nblk; ++n, ++g) {
+          const int s = g % BW_STAGES;
+          if (!mbar_wait(&qd_full[s], (g / BW_STAGES) & 1u) || (g >= 1 && !mbar_wait(s_free, (g - 1) & 1u))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
+          const uint32_t doa = qa + TILE;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          tc_mma(tmem + DKV_T_S, make_sdesc(ka + kk * 32, 0), make_sdesc(qa + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
-          tc_mma(tmem + DKV_T_DP, make_sdesc(va + kk * 32, 0), make_sdesc(doa + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            tc_mma(tmem + DKV_T_S, make_sdesc(ka + kk * 32, 0), make_sdesc(qa + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
+            tc_mma(tmem + DKV_T_DP, make_sdesc(va + kk * 32, 0), make_sdesc(doa + kk * 32, 0), id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full);
+          if (n == nblk - 1) tc_commit(&kv_empty[kvb]);
+          if (g >= 1 && !acc_step(g - 1, pn, plast)) {
+            ok = false;
+            break;
+          }
+          pn = n;
+          plast = n == nblk - 1;
         }
-        tc_commit(s_full);
-        if (n >= 1 && !acc_step(n - 1)) ok = false;
       }
-      if (ok && nblk > 0 && !acc_step(nblk - 1)) ok = false;
+      if (ok && g >= 1 && !acc_step(g - 1, pn, plast)) ok = false;
       if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
-      tc_commit(acc_done);
-      if (!mbar_wait_drain(acc_done, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_commit(drain);
+      if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
     }
   } else {
     // ---------------------------------------------------- compute warps
     const int qw = warp & 3;
-    const int hf = (warp - 2) >> 2;  // which 64 queries of the 128-query tile
+    const int cq = (warp - 2) >> 2;  // which 32 queries of the 128-query tile (and 16 dK/dV columns)
     const int kr = qw * 32 + lane;   // key row within the block
-    const int key = kb * BT + kr;    // key position
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+    uint32_t g = 0, t = 0;
     bool ok = true;
-    for (int n = 0; n < nblk; ++n) {
-      const int i = kb + n, s = n % BW_STAGES;
-      if (!warp_wait(s_full, n & 1u) || !warp_wait(&qd_full[s], (n / BW_STAGES) & 1u)) {
+    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      int kb, bh;
+      item(w, kb, bh);
+      const int b = bh / H, h = bh % H, row0 = b * T;
+      const int nblk = nqb - kb;
+      const int key = kb * BT + kr;  // key position
+      for (int n = 0; n < nblk; ++n, ++g) {
+        const int i = kb + n, s = g % BW_STAGES;
+        if (!warp_wait(s_full, g & 1u) || !warp_wait(&qd_full[s], (g / BW_STAGES) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tl + DKV_T_S + cq * 32, sv);
+        tmem_ld32(tl + DKV_T_DP + cq * 32, dv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        const int q0 = i * BT + cq * 32;          // first query of this warp's columns
+        const bool diag = q0 < kb * BT + BT - 1;  // some query of the columns precedes some key
+        const float* ldl =
+            reinterpret_cast<const float*>(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES + 2 * TILE) + cq * 32;
+        // P^T and dS^T of this block, packed to bf16 pairs in place
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          const float4 la = *reinterpret_cast<const float4*>(ldl + c);
+          const float4 lb = *reinterpret_cast<const float4*>(ldl + c + 4);
+          const float4 da = *reinterpret_cast<const float4*>(ldl + BT + c);
+          const float4 db = *reinterpret_cast<const float4*>(ldl + BT + c + 4);
+          const float l8[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+          const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          float p[8], ds[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float a = fmaf(__uint_as_float(sv[c + e]), sl2, -l8[e]);
+            float pe = (EX2_FMA_EVERY > 0 && ((c + e) / 2) % (EX2_FMA_EVERY > 0 ? EX2_FMA_EVERY : 1) ==
+                                                  (EX2_FMA_EVERY > 0 ? EX2_FMA_EVERY : 1) - 1)
+                           ? ex2_fma(a)
+                           : ex2f(a);
+            if (diag && (q0 + c + e < key)) pe = 0.f;
+            p[e] = pe;
+            ds[e] = pe * (__uint_as_float(dv[c + e]) - d8[e]);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            sv[(c >> 1) + e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+            dv[(c >> 1) + e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
+          }
+        }
+        // the previous step's dV / dK MMAs have read P^T and dS^T
+        if (g >= 1 && !warp_wait(p_free, (g - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tl + DKV_T_P + cq * 16, sv);
+        tmem_st16(tl + DKV_T_DS + cq * 16, dv);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      // item epilogue: dV, dK (scaled) and their column sums.  The next item's
+      // first dV / dK MMAs overwrite the accumulators; they wait for that
+      // item's first P^T / dS^T, which these warps write only after the loads
+      // below.
+      if (!warp_wait(acc_done, t & 1u)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[64], dv[64];
-      tmem_ld64(tl + DKV_T_S + hf * 64, sv);
-      tmem_ld64(tl + DKV_T_DP + hf * 64, dv);
+      uint32_t av[16], ak[16];
+      tmem_ld16(tl + DKV_T_DV + cq * 16, av);
+      tmem_ld16(tl + DKV_T_DK + cq * 16, ak);
       tmem_wait_ld();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      const int q0 = i * BT + hf * 64;                // first query of this warp's columns
-      const bool diag = q0 < kb * BT + BT - 1;        // some query of the columns precedes some key
-      const float* ldl =
-          reinterpret_cast<const float*>(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES + 2 * TILE) + hf * 64;
-      // P^T and dS^T of this block, packed to bf16 pairs in place
+      if (key < T) {
+        store_row16(dqkv + ((long)row0 + key) * (3L * C) + 2 * C + h * HD + cq * 16, av, 1.f);
+        store_row16(dqkv + ((long)row0 + key) * (3L * C) + C + h * HD + cq * 16, ak, scale);
+      }
+      if (colsum) {
+        float cs[16];
+        const long prow = (((long)b * nqb + kb) * 4 + qw) * (3L * C);
 #pragma unroll
-      for (int c = 0; c < 64; c += 8) {
-        const float4 la = *reinterpret_cast<const float4*>(ldl + c);
-        const float4 lb = *reinterpret_cast<const float4*>(ldl + c + 4);
-        const float4 da = *reinterpret_cast<const float4*>(ldl + BT + c);
-        const float4 db = *reinterpret_cast<const float4*>(ldl + BT + c + 4);
-        const float l8[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-        const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-        float p[8], ds[8];
+        for (int i = 0; i < 16; ++i) cs[i] = key < T ? __uint_as_float(ak[i]) * scale : 0.f;
+        const float tk = warp_colsum16(cs, lane);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float pe = ex2f(fmaf(__uint_as_float(sv[c + e]), sl2, -l8[e]));
-          if (diag && (q0 + c + e < key)) pe = 0.f;
-          p[e] = pe;
-          ds[e] = pe * (__uint_as_float(dv[c + e]) - d8[e]);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          sv[(c >> 1) + e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
-          dv[(c >> 1) + e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
+        for (int i = 0; i < 16; ++i) cs[i] = key < T ? __uint_as_float(av[i]) : 0.f;
+        const float tv = warp_colsum16(cs, lane);
+        if (lane < 16) {
+          colsum[prow + C + h * HD + cq * 16 + lane] = tk;
+          colsum[prow + 2 * C + h * HD + cq * 16 + lane] = tv;
         }
       }
-      // the previous block's dV / dK MMAs have read P^T and dS^T
-      if (n >= 1 && !warp_wait(p_free, (n - 1) & 1u)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st32(tl + DKV_T_P + hf * 32, sv);
-      tmem_st32(tl + DKV_T_DS + hf * 32, dv);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    float cv[32], ck[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) cv[i] = ck[i] = 0.f;
-    if (ok && warp_wait(acc_done, 0)) {
-      tc_fence_after();
-      uint32_t a[32];
-      tmem_ld32(tl + DKV_T_DV + hf * 32, a);
-      tmem_wait_ld();
-      if (key < T) {
-        store_row32(dqkv + ((long)row0 + key) * (3L * C) + 2 * C + h * HD + hf * 32, a, 1.f);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) cv[i] = __uint_as_float(a[i]);
-      }
-      tmem_ld32(tl + DKV_T_DK + hf * 32, a);
-      tmem_wait_ld();
-      if (key < T) {
-        store_row32(dqkv + ((long)row0 + key) * (3L * C) + C + h * HD + hf * 32, a, scale);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ck[i] = __uint_as_float(a[i]) * scale;
-      }
-    } else {
-      ok = false;
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
-    if (colsum) {
-      red[(hf * 4 + qw) * 32 + lane] = warp_colsum32(ck, lane);
-      red[256 + (hf * 4 + qw) * 32 + lane] = warp_colsum32(cv, lane);
-    }
   }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BW_TMEM_COLS) : "memory");
-  }
-  // column sums of dK and dV over the block's rows (the key and value bias
-  // gradients), one partial row per 128-row block, quarters in a fixed order
-  if (colsum && warp >= 2 && warp < 6) {
-    const int kv = (warp - 2) >> 1, hf = (warp - 2) & 1;  // kv 0: dK, 1: dV
-    const float* rr = red + kv * 256 + hf * 128;
-    const float t = ((rr[lane] + rr[32 + lane]) + rr[64 + lane]) + rr[96 + lane];
-    colsum[((long)b * nqb + kb) * (3L * C) + (1 + kv) * C + h * HD + hf * 32 + lane] = t;
   }
 }
 
@@ -548,12 +709,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
 static inline long backward_scratch_floats(int B, int T, int H) {
   return (long)B * H * ((T + BT - 1) / BT) * LD_FLOATS;
 }
+// rows of the column-sum partials: one per (batch, 128-row block, lane quarter)
+static inline long backward_colsum_rows(int B, int T) { return (long)B * ((T + BT - 1) / BT) * 4; }
 
 // dq_kernel first (it also writes lse*log2(e) and D into `ld`), then
 // dkdv_kernel.  ld: fp32 scratch of backward_scratch_floats(B, T, H) elements,
-// 16-byte aligned.  colsum (may be null): [B * ceil(T/128)][3C] fp32 partial
-// column sums of dqkv, one row per 128-row block of each batch (summing them
-// over the rows gives the qkv bias gradient).
+// 16-byte aligned.  colsum (may be null): [backward_colsum_rows(B, T)][3C]
+// fp32 partial column sums of dqkv (summing them over the rows gives the qkv
+// bias gradient).
 static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, bf16* dqkv,
                                    float* ld, int B, int T, int H, cudaStream_t st, float* colsum = nullptr) {
   static DeviceOnce once;
@@ -570,9 +733,10 @@ static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16*
   if (make_tmap(&td, dout, C, (long)B * T, C, 64, BT) != 0) return cudaErrorInvalidValue;
   const float scale = 1.f / sqrtf((float)HD);
   const float sl2 = 1.4426950408889634f * scale;
-  dim3 grid((T + BT - 1) / BT, B * H);
-  dq_kernel<<<grid, BW_THREADS, DQ_SMEM, st>>>(tq, td, out, lse, ld, dqkv, colsum, T, H, scale, sl2);
-  dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, T, H, scale, sl2);
+  const int items = ((T + BT - 1) / BT) * B * H;
+  const int grid = items < num_sms_attn() ? items : num_sms_attn();
+  dq_kernel<<<grid, BW_THREADS, DQ_SMEM, st>>>(tq, td, out, lse, ld, dqkv, colsum, T, H, B * H, scale, sl2);
+  dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, T, H, B * H, scale, sl2);
   return cudaGetLastError();
 }
 

@@ -5,6 +5,7 @@
 #include "attention_tc.cuh"
 #include "attention_tc_bwd.cuh"
 #include "model_pass.cuh"
+#include "model_decode.cuh"
 
 #include <mutex>
 
@@ -60,6 +61,12 @@ void gpt2_destroy(gpt2_t* h) {
   for (auto& g : h->graphs)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  if (h->side_stream) {
+    cudaStreamSynchronize(h->side_stream);
+    cudaStreamDestroy(h->side_stream);
+  }
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_sorted) cudaEventDestroy(h->ev_sorted);
   if (h->ev_in) cudaEventDestroy(h->ev_in);
   if (h->ev_out) cudaEventDestroy(h->ev_out);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
@@ -386,6 +393,32 @@ int gpt2_set_wait_limit_ns(uint64_t limit_ns) {
   if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) {
     cudaGetLastError();
     return GPT2_ECUDA;
+  }
+  return GPT2_OK;
+}
+
+int gpt2_prefill(gpt2_t* h, const int32_t* d_tokens, int B, int T0, float temperature, int top_k, uint64_t seed,
+                 int32_t* d_next) {
+  if (h == nullptr) return GPT2_EINVAL;
+  return prefill_impl(h, d_tokens, B, T0, temperature, top_k, seed, d_next);
+}
+
+int gpt2_decode_step(gpt2_t* h, const int32_t* d_tokens, int B, int pos, float temperature, int top_k, uint64_t seed,
+                     int32_t* d_next) {
+  if (h == nullptr) return GPT2_EINVAL;
+  return decode_impl(h, d_tokens, B, pos, temperature, top_k, seed, d_next);
+}
+
+int gpt2_get_decode_logits(gpt2_t* h, float* dst) {
+  if (h == nullptr || dst == nullptr) return GPT2_EINVAL;
+  if (h->gen_B == 0) return set_err(h, GPT2_ESTATE, "no prefill yet");
+  RET_IF(check_device_flags(h));
+  const size_t n = (size_t)h->gen_B * h->Vp;
+  std::vector<uint16_t> tmp(n);
+  CU_CHECK(h, cudaMemcpy(tmp.data(), h->dec_logits, n * 2, cudaMemcpyDeviceToHost));
+  for (size_t i = 0; i < n; ++i) {
+    const uint32_t u = (uint32_t)tmp[i] << 16;
+    memcpy(dst + i, &u, 4);
   }
   return GPT2_OK;
 }

@@ -78,6 +78,14 @@ struct gpt2 {
   // state of the last forward
   int B = 0, T = 0;
   bool have_fwd = false, have_targets = false, logits_valid = false, have_bwd_keys = false;
+
+  // generation (bf16 mode): KV cache [L][max_B][block][2C] (k then v) and the
+  // per-step activations of up to max_B sequences, allocated on first use
+  bf16* kv = nullptr;
+  float *dec_x = nullptr, *dec_mean = nullptr, *dec_rstd = nullptr;
+  bf16 *dec_ln = nullptr, *dec_qkv = nullptr, *dec_att = nullptr, *dec_u = nullptr, *dec_a = nullptr;
+  bf16* dec_logits = nullptr;  // [max_B, Vp] logits of the last prefill / decode step
+  int gen_B = 0, gen_len = 0;  // sequences and positions held in the cache
   const int32_t* last_tok = nullptr;
   const int32_t* last_tgt = nullptr;
 
@@ -93,6 +101,10 @@ struct gpt2 {
   bool use_graphs = true;
   cudaStream_t cap_stream = nullptr;
   cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+  // the embedding backward's key sort runs beside the forward on side_stream
+  cudaStream_t side_stream = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_sorted = nullptr;
+  bool sort_pending = false;
 
   // opt-in per-class device timing (measurement support)
   bool timing = false;
@@ -202,7 +214,8 @@ static void free_all(gpt2* h) {
                   h->ce_lse,  h->losses,  h->d_loss,   h->argmax,   h->dres,     h->dln,      h->attn_D,
                   h->ln_part, h->cs_part, h->dres_bf,  h->dbig,     h->dqkv,     h->datt,     h->splitk_ws,
                   h->emb_keys, h->emb_part, h->normbuf, h->d_step, h->norm_part, h->segs,    h->d_bad,    h->tok_dev,
-                  h->tgt_dev, h->ce_part, h->attn_cs};
+                  h->tgt_dev, h->ce_part, h->attn_cs, h->kv, h->dec_x, h->dec_mean, h->dec_rstd, h->dec_ln,
+                  h->dec_qkv, h->dec_att, h->dec_u, h->dec_a, h->dec_logits};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }

@@ -114,7 +114,7 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   ALLOC(h, h->ce_lse, (size_t)Mx * 4);
   if (h->prec == GPT2_BF16) {
     ALLOC(h, h->ce_part, (size_t)Mx * tcg::ce_halves(h->Vp) * 3 * 4);
-    ALLOC(h, h->attn_cs, (size_t)h->maxB * ((h->maxT + 127) / 128) * 3 * C * 4);
+    ALLOC(h, h->attn_cs, (size_t)tcfa::backward_colsum_rows(h->maxB, h->maxT) * 3 * C * 4);
   }
   ALLOC(h, h->losses, (size_t)Mx * 4);
   ALLOC(h, h->d_loss, 16);
@@ -189,6 +189,9 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
     CU_CHECK(h, cudaFuncSetAttribute(k::ce_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_smem));
   CU_CHECK(h, cudaFuncSetAttribute(k::sort_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, h->sort_cap * 4));
   CU_CHECK(h, cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+  CU_CHECK(h, cudaStreamCreateWithFlags(&h->side_stream, cudaStreamNonBlocking));
+  CU_CHECK(h, cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+  CU_CHECK(h, cudaEventCreateWithFlags(&h->ev_sorted, cudaEventDisableTiming));
   CU_CHECK(h, cudaEventCreateWithFlags(&h->ev_in, cudaEventDisableTiming));
   CU_CHECK(h, cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming));
   CU_CHECK(h, cudaStreamSynchronize(h->stream));

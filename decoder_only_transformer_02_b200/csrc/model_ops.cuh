@@ -241,7 +241,7 @@ static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
 // grads[boff .. +3C] += the attention backward's per-block column sums of dqkv
 static int op_attn_bias_reduce(gpt2* h, size_t boff) {
   KTimer kt(h, KC_OTHER, 0.0, 0.0);
-  const int nblk = h->B * ((h->T + 127) / 128);
+  const int nblk = (int)tcfa::backward_colsum_rows(h->B, h->T);
   const int n = 3 * h->C;
   k::partials_reduce_kernel<<<(n + 31) / 32, 256, 0, h->stream>>>(h->attn_cs, nblk, n, n, h->G32(boff), nullptr,
                                                                   nullptr);

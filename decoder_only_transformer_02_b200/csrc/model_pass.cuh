@@ -41,6 +41,19 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
   if (tgt && tgt != h->tgt_dev)
     CU_CHECK(h, cudaMemcpyAsync(h->tgt_dev, tgt, M * 4, cudaMemcpyDeviceToDevice, h->stream));
   const int32_t* dtgt = tgt ? h->tgt_dev : nullptr;
+  if (dtgt != nullptr && !h->timing) {
+    // the embedding backward's (token, position) sort needs only the ids: run
+    // it on the side stream while the forward runs; the backward joins it
+    CU_CHECK(h, cudaEventRecord(h->ev_fork, h->stream));
+    CU_CHECK(h, cudaStreamWaitEvent(h->side_stream, h->ev_fork, 0));
+    k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->side_stream>>>(h->tok_dev, (int)M, h->Vp,
+                                                                               h->emb_keys, h->sort_cap);
+    LAUNCH_CHECK(h);
+    CU_CHECK(h, cudaEventRecord(h->ev_sorted, h->side_stream));
+    h->sort_pending = true;
+  } else {
+    h->sort_pending = false;
+  }
 
   {
     KTimer kt(h, KC_EMB, 0.0, 12.0 * M * C);
@@ -143,9 +156,14 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
   }
   // embeddings: dwte[tok] += dx0 (sorted, fixed order), dwpe[t] += sum_b dx0[b, t]
   KTimer kt(h, KC_EMB, 0.0, 8.0 * M * C + 8.0 * T * C);
-  k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->stream>>>(h->tok_dev, (int)M, h->Vp, h->emb_keys,
-                                                                        h->sort_cap);
-  LAUNCH_CHECK(h);
+  if (h->sort_pending) {
+    CU_CHECK(h, cudaStreamWaitEvent(h->stream, h->ev_sorted, 0));
+    h->sort_pending = false;
+  } else {
+    k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->stream>>>(h->tok_dev, (int)M, h->Vp, h->emb_keys,
+                                                                          h->sort_cap);
+    LAUNCH_CHECK(h);
+  }
   const int eth = C < 256 ? C : 256;
   k::embed_bwd_partial_kernel<<<(unsigned)((M + k::EMB_CH - 1) / k::EMB_CH), eth, 0, h->stream>>>(
       h->emb_keys, h->dres, (int)M, C, h->emb_part);

@@ -339,15 +339,64 @@ __device__ __forceinline__ void epi_ce_chunk(const Params& p, int row, int col0,
   softmax_stats_merge(m, s, mi, cm, (cs[0] + cs[1]) + (cs[2] + cs[3]), ci);
 }
 
+// Fused math on 32 columns whose residual / accumulator (fp32, 4 x 32-byte
+// words) or GELU pre-activation (bf16, 2 x 32-byte words) the caller already
+// loaded into x: the vectorised epilogue of EPI_RESID_F32, EPI_ACCUM_F32 and
+// EPI_DGELU.
+__device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int col0, const uint32_t (&r)[32],
+                                                 const uint32_t (*x)[8]) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  const long base = (long)row * p.ldc + col0;
+  if (p.epi == EPI_DGELU) {
+    bf16* o = reinterpret_cast<bf16*>(p.out) + base;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float2 f = unpack_bf16x2(x[hh][e]);
+        v[16 * hh + 2 * e] *= gelu_tanh_grad<true>(f.x);
+        v[16 * hh + 2 * e + 1] *= gelu_tanh_grad<true>(f.y);
+      }
+    st_bf16x16(o, v);
+    st_bf16x16(o + 16, v + 16);
+    return;
+  }
+  if (p.bias != nullptr && p.epi == EPI_RESID_F32) {
+    const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 bb = __ldg(b4 + i);
+      v[4 * i] += bb.x;
+      v[4 * i + 1] += bb.y;
+      v[4 * i + 2] += bb.z;
+      v[4 * i + 3] += bb.w;
+    }
+  }
+  float* o = reinterpret_cast<float*>(p.out) + base;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[8 * i + e] += __uint_as_float(x[i][e]);
+    st_f32x8(o + 8 * i, v + 8 * i);
+  }
+}
+
 // The epilogue of one accumulator tile for one warp: its TMEM lane quarter
 // (rows `row` of the tile, one per lane) and its half of the columns
-// [cbase, cbase + BN/2).  release() hands the accumulator buffer back to the
-// MMA issuer once the warp's last columns are in registers (called by lane 0).
-template <int BN, bool CE, class Release>
-__device__ __forceinline__ void epilogue_tile(const Params& p, int row, int nb, int split, uint32_t tbase, int cbase,
-                                              int whalf, int lane, Release release) {
+// [cbase, cbase + BN/2).  wait_acc() waits for the accumulator (false: gave
+// up); release() hands the accumulator buffer back to the MMA issuer once the
+// warp's last columns are in registers (called by lane 0).  The epilogues that
+// read memory (residual, accumulator, GELU pre-activation) issue a chunk's
+// loads before they wait for its accumulator columns, the first chunk's even
+// before the accumulator is complete.  Returns false when wait_acc gave up.
+template <int BN, bool CE, class Wait, class Release>
+__device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, int split, uint32_t tbase, int cbase,
+                                              int whalf, int lane, Wait wait_acc, Release release) {
   constexpr int CHUNKS = BN / 64 / (EPI_WARPS / 4);  // 64-column chunks per warp
   if constexpr (CE) {
+    if (!wait_acc()) return false;
     // logits and their per-(row, half tile) softmax statistics
     float m = -INFINITY, s = 0.f;
     int mi = 0x7fffffff;
@@ -372,31 +421,55 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, int row, int nb, 
       cp[2] = __int_as_float(mi);
     }
   } else {
+    const bool f32_in = p.epi == EPI_RESID_F32 || p.epi == EPI_ACCUM_F32;
+    const bool loads = (f32_in || p.epi == EPI_DGELU) && p.vec32 && row < p.M;
     // 64 accumulator columns per TMEM wait; the buffer is handed back to the
     // MMA warp as soon as its last columns are in registers
 #pragma unroll 1
     for (int j = 0; j < CHUNKS; ++j) {
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tbase + cbase + j * 64, r0);
-      tmem_ld32(tbase + cbase + j * 64 + 32, r1);
-      tmem_wait_ld();
-      if (j == CHUNKS - 1) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) release();
+      const int col = nb * BN + cbase + j * 64;
+      const bool pre = loads && col + 64 <= p.N;
+      uint32_t x[8][8];
+      if (pre) {
+        if (f32_in) {
+          const float* src = (p.epi == EPI_RESID_F32 ? p.resid : reinterpret_cast<const float*>(p.out)) +
+                             (long)row * p.ldc + col;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ld32(src + 8 * i, x[i]);
+        } else {
+          const bf16* src = p.aux + (long)row * p.ldc + col;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ld32(src + 16 * i, x[i]);
+        }
       }
+      if (j == 0 && !wait_acc()) return false;
+      // the chunk's two 32-column halves, one TMEM load and wait each
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int col0 = nb * BN + cbase + j * 64 + h * 32;
-        if (row < p.M && col0 < p.N) {
-          if (col0 + 32 <= p.N && p.vec32)
-            epi_store<true>(p, row, col0, split, h ? r1 : r0);
+        uint32_t r[32];
+        tmem_ld32(tbase + cbase + j * 64 + 32 * h, r);
+        tmem_wait_ld();
+        if (j == CHUNKS - 1 && h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release();
+        }
+        const int col0 = col + h * 32;
+        if (pre) {
+          if (f32_in)
+            epi_store_loaded(p, row, col0, r, &x[4 * h]);
           else
-            epi_store<false>(p, row, col0, split, h ? r1 : r0);
+            epi_store_loaded(p, row, col0, r, &x[2 * h]);
+        } else if (row < p.M && col0 < p.N) {
+          if (col0 + 32 <= p.N && p.vec32)
+            epi_store<true>(p, row, col0, split, r);
+          else
+            epi_store<false>(p, row, col0, split, r);
         }
       }
     }
   }
+  return true;
 }
 
 // --------------------------------------------------------------- kernel
@@ -544,15 +617,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       int mb, nb, split;
       decode_tile(p, tile, mb, nb, split);
       const uint32_t buf = tc & 1u;
-      if (!mbar_wait(&tfull[buf], (tc >> 1) & 1u)) {
+      const int row = mb * BM + q * 32 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      const bool ok = epilogue_tile<BN, CE>(
+          p, row, nb, split, tbase, cbase, (warp - 2) >> 2, lane,
+          [&] {
+            const bool got = mbar_wait(&tfull[buf], (tc >> 1) & 1u);
+            tc_fence_after();
+            return got;
+          },
+          [&] { mbar_arrive(&tempty[buf]); });
+      if (!ok) {
         set_device_err(DERR_WAIT_TIMEOUT);
         break;
       }
-      tc_fence_after();
-      const int row = mb * BM + q * 32 + lane;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      epilogue_tile<BN, CE>(p, row, nb, split, tbase, cbase, (warp - 2) >> 2, lane,
-                            [&] { mbar_arrive(&tempty[buf]); });
     }
   }
   __syncthreads();
@@ -787,16 +865,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int mb, nb, split;
       decode_tile(p, tile, mb, nb, split);
       const uint32_t buf = tc & 1u;
-      if (!mbar_wait(&tfull[buf], (tc >> 1) & 1u)) {
-        set_device_err(DERR_WAIT_TIMEOUT);
-        break;
-      }
-      tc_fence_after();
       const int row = mb * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
       const uint32_t tempty_leader = mapa_rank(smem_u32(&tempty[buf]), 0);
-      epilogue_tile<BN, CE>(p, row, nb, split, tbase, cbase, (warp - 2) >> 2, lane,
-                            [&] { mbar_arrive_cluster(tempty_leader); });
+      const bool ok = epilogue_tile<BN, CE>(
+          p, row, nb, split, tbase, cbase, (warp - 2) >> 2, lane,
+          [&] {
+            const bool got = mbar_wait(&tfull[buf], (tc >> 1) & 1u);
+            tc_fence_after();
+            return got;
+          },
+          [&] { mbar_arrive_cluster(tempty_leader); });
+      if (!ok) {
+        set_device_err(DERR_WAIT_TIMEOUT);
+        break;
+      }
     }
   }
   __syncthreads();
@@ -890,15 +973,12 @@ static cudaError_t launch2(const CUtensorMap& ta, const CUtensorMap& tb, const P
 }
 
 // Which kernel serves a shape: the 2-SM pair kernel for N > 128 with more
-// than 128 rows when GPT2_GEMM_2SM=1 is set in the environment, else the 1-SM
-// kernel.
+// than 128 rows, unless GPT2_GEMM_2SM=0 is set in the environment (then the
+// 1-SM kernel serves every shape; read at each call, for comparisons).
 static bool use_pair_kernel(int M, int N, int bn) {
-  static int mode = -1;
-  if (mode < 0) {
-    const char* e = getenv("GPT2_GEMM_2SM");
-    mode = (e != nullptr && e[0] == '1') ? 1 : 0;
-  }
-  return mode == 1 && bn == 256 && M > BM && N > 128;
+  const char* e = getenv("GPT2_GEMM_2SM");
+  const bool pair = !(e != nullptr && e[0] == '0');
+  return pair && bn == 256 && M > BM && N > 128;
 }
 
 int choose_splits(int tiles, int kb_total, int units) {

@@ -28,6 +28,7 @@ EXPORTED = [
     "gpt2_last_error", "gpt2_attention_forward", "gpt2_attention_backward", "gpt2_attention_workspace_floats",
     "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes", "gpt2_set_timing", "gpt2_get_timing",
     "gpt2_attention_backward_noalloc", "gpt2_set_graphs", "gpt2_check_device_error", "gpt2_set_wait_limit_ns",
+    "gpt2_prefill", "gpt2_decode_step", "gpt2_get_decode_logits",
 ]
 ATTN_NOALLOC_MAX_ROWS = 1 << 19  # padded (batch, head, position) rows
 KCLASSES = ["matmul", "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd", "cross_entropy",
@@ -94,6 +95,9 @@ def load_library():
         "gpt2_set_graphs": (I, [P, I]),
         "gpt2_check_device_error": (I, [P]),
         "gpt2_set_wait_limit_ns": (I, [ctypes.c_uint64]),
+        "gpt2_prefill": (I, [P, P, I, I, F, I, ctypes.c_uint64, P]),
+        "gpt2_decode_step": (I, [P, P, I, I, F, I, ctypes.c_uint64, P]),
+        "gpt2_get_decode_logits": (I, [P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -215,6 +219,24 @@ class GPT2:
 
     def set_graphs(self, enable: bool):
         self._check(self._lib.gpt2_set_graphs(self._h, 1 if enable else 0))
+
+    # -- generation
+    def prefill(self, tokens, next_out, temperature=1.0, top_k=1, seed=0):
+        """tokens: device int32 [B, T0]; next_out: device int32 [B] (receives
+        the token at position T0)."""
+        B, T0 = tokens.shape
+        self._check(self._lib.gpt2_prefill(self._h, _ptr(tokens), B, T0, temperature, top_k, seed, _ptr(next_out)))
+
+    def decode_step(self, tokens, pos, next_out, temperature=1.0, top_k=1, seed=0):
+        """tokens: device int32 [B] at position pos; next_out: device int32 [B]."""
+        B = tokens.shape[0]
+        self._check(self._lib.gpt2_decode_step(self._h, _ptr(tokens), B, pos, temperature, top_k, seed,
+                                               _ptr(next_out)))
+
+    def get_decode_logits(self, B) -> np.ndarray:
+        a = np.empty((B, self.cfg.padded_vocab), dtype=np.float32)
+        self._check(self._lib.gpt2_get_decode_logits(self._h, a.ctypes.data))
+        return a
 
     # -- measurement support
     def set_timing(self, enable: bool):

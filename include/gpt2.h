@@ -127,6 +127,34 @@ int gpt2_train_step(gpt2_t* h, const int32_t* h_tokens, const int32_t* h_targets
  * Scratch: Building GPT-2", Training Setup: 715 warmup steps, 19073 iterations). */
 double gpt2_lr_at(int it, double max_lr, double min_lr, int warmup, int max_steps);
 
+/* ---- generation (forward only, KV cache; bf16 mode) ----
+ * "Let's reproduce GPT-2 (124M)", Chapters: sampling init, prefix tokens;
+ * sampling loop.  The model continues B prefixes of equal length one token
+ * at a time.  The cache holds every layer's keys and values for up to
+ * block_size positions of max_B sequences (allocated by the first prefill:
+ * n_layer * max_B * block_size * 2 * n_embd bf16).
+ * Next-token rule: top-k sampling from softmax(logits / temperature) over the
+ * top_k largest logits of the real vocabulary [0, vocab_size) (ties at the
+ * k-th place to the lower id); top_k = 1 or temperature = 0 is the greedy
+ * argmax.  The uniform draw of sequence b for the token at position p is the
+ * top 53 bits of splitmix64(seed * 2^32 + p * 2^16 + b), where splitmix64 is
+ * the generator of Steele, Lea and Flood (OOPSLA 2014), so every draw is
+ * reproducible.  1 <= top_k <= 64; GPT2_EINVAL otherwise or in FP32 mode.
+ * d_next: device int32 [B] that receives the next token of every sequence. */
+/* Run the forward on d_tokens [B, T0] (T0 <= max_T), fill the cache with
+ * positions 0..T0-1 and sample the token at position T0 from the last
+ * position's logits.  Replaces whatever the cache held. */
+int gpt2_prefill(gpt2_t* h, const int32_t* d_tokens, int B, int T0, float temperature, int top_k, uint64_t seed,
+                 int32_t* d_next);
+/* One step: d_tokens [B] are the tokens at position pos, which must equal the
+ * number of positions the cache holds (T0 after the prefill, +1 per step) and
+ * be below block_size; B must be the prefill's.  Appends their keys and values
+ * to the cache and samples the token at position pos + 1. */
+int gpt2_decode_step(gpt2_t* h, const int32_t* d_tokens, int B, int pos, float temperature, int top_k,
+                     uint64_t seed, int32_t* d_next);
+/* [B, Vp] logits (as fp32) from which the last prefill or decode step drew. */
+int gpt2_get_decode_logits(gpt2_t* h, float* h_dst);
+
 /* ---- accessors (parity checks, checkpoint / resume); all synchronise ---- */
 int64_t gpt2_num_params(const gpt2_t* h);
 int gpt2_get_params(gpt2_t* h, float* h_dst);       /* fp32 master weights, flat order */

@@ -447,3 +447,57 @@ def train_step(params, m, v, t, cfg: Config, micro_batches, lr, **adamw_kw):
         losses.append(st["loss"])
     p, m, v, norm = adamw_step(params, grads, m, v, t, lr, cfg, **adamw_kw)
     return p, m, v, float(np.mean(losses)), norm
+
+
+# --------------------------------------------------------------------------
+# generation
+# --------------------------------------------------------------------------
+# [C] chapters "sampling init, prefix tokens, tokenization", "sampling loop":
+# the model continues a prefix one token at a time, each new token drawn from
+# the distribution its logits give at the last position.  The pages name no
+# sampling rule.  reading: top-k sampling from softmax(logits / temperature)
+# over the k largest logits of the real vocabulary [0, V) (padded ids are not
+# tokens), ties at the k-th place going to the lower id; k = 1 (or
+# temperature 0) is the greedy argmax.  What KV caching changes is only how
+# the logits are computed: the reference for the logits at position t is
+# forward() on the prefix tokens[:t+1], whose last row they are.
+
+_SM64_GAMMA = 0x9E3779B97F4A7C15
+_MASK64 = (1 << 64) - 1
+
+
+def splitmix64(x: int) -> int:
+    """The splitmix64 generator's output function (Steele, Lea and Flood,
+    "Fast splittable pseudorandom number generators", OOPSLA 2014): add the
+    golden-ratio increment, then two xor-shift-multiply rounds and a final
+    xor-shift, all modulo 2^64."""
+    z = (x + _SM64_GAMMA) & _MASK64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK64
+    return z ^ (z >> 31)
+
+
+def sample_uniform(seed: int, row: int, pos: int) -> float:
+    """Counter-based uniform in [0, 1) for sequence `row` at position `pos`:
+    the top 53 bits of splitmix64(seed * 2^32 + pos * 2^16 + row).
+    reading: the pages fix no generator; this one is defined here and in the
+    device sampler alike, so both draw the same u."""
+    key = ((seed & 0xFFFFFFFF) << 32 | (pos & 0xFFFF) << 16 | (row & 0xFFFF)) & _MASK64
+    return (splitmix64(key) >> 11) * (1.0 / (1 << 53))
+
+
+def sample_next(logits_row, vocab: int, temperature: float, top_k: int, u: float) -> int:
+    """One draw of the next token from one row of logits (see the reading
+    above): keep the top_k largest logits among ids [0, vocab), form
+    p_i = exp((z_i - z_max) / temperature) / sum, and return the first id (in
+    descending-logit order) whose cumulative probability exceeds u."""
+    z = np.asarray(logits_row, dtype=np.float64)[:vocab]
+    if top_k <= 1 or temperature <= 0.0:
+        return int(np.argmax(z))
+    k = min(top_k, vocab)
+    order = np.lexsort((np.arange(vocab), -z))[:k]  # descending logit, lower id first on ties
+    zk = z[order]
+    p = np.exp((zk - zk[0]) / temperature)
+    cdf = np.cumsum(p) / p.sum()
+    i = int(np.searchsorted(cdf, u, side="right"))
+    return int(order[min(i, k - 1)])

@@ -18,6 +18,17 @@ def _lib():
     return G
 
 
+@pytest.fixture(params=["pair", "single"], autouse=True)
+def kernel(request, monkeypatch):
+    """Run every case on both GEMM kernels: the 2-SM pair kernel (the default
+    for N > 128 and M > 128) and the 1-SM kernel (GPT2_GEMM_2SM=0)."""
+    if request.param == "single":
+        monkeypatch.setenv("GPT2_GEMM_2SM", "0")
+    else:
+        monkeypatch.delenv("GPT2_GEMM_2SM", raising=False)
+    return request.param
+
+
 def _operands(M, N, K, seed):
     from decoder_only_transformer_02_b200.synthetic import normal_array
     A = bf16_round(normal_array((M, K), seed))        # logical A[m, k]

@@ -360,3 +360,58 @@ def test_planted_oracle_mistakes_are_caught(monkeypatch, mistake):
     ok = (np.allclose(st["logits"], logits.detach().numpy(), rtol=1e-8, atol=1e-10)
           and np.allclose(g, TR.flatten_grads(p, cfg), rtol=1e-6, atol=1e-10))
     assert not ok
+
+
+# ------------------------------------------------------------- generation
+
+def test_splitmix64_published_sequence():
+    """The generator's output for a sequence seeded with 1234567 (state
+    advanced by the golden-ratio increment per draw), as printed with the
+    reference C implementation of splitmix64."""
+    s, g = 1234567, O._SM64_GAMMA
+    got = [O.splitmix64((s + i * g) & O._MASK64) for i in range(5)]
+    assert got == [6457827717110365317, 3203168211198807973, 9817491932198370423, 4593380528125082431,
+                   16408922859458223821]
+
+
+def test_sample_uniform_range_and_spread():
+    u = np.array([O.sample_uniform(7, b, p) for b in range(16) for p in range(256)])
+    assert np.all((u >= 0) & (u < 1))
+    assert abs(u.mean() - 0.5) < 0.02 and abs(u.var() - 1 / 12) < 0.01
+    assert len(set(u.tolist())) == u.size
+
+
+def test_sample_next_greedy_and_edges():
+    rng = np.random.default_rng(3)
+    z = rng.normal(0, 2, 64)
+    V = 60           # ids 60..63 are padding and never drawn
+    z[61] = 100.0
+    best = int(np.argmax(z[:V]))
+    assert O.sample_next(z, V, 1.0, 1, 0.7) == best
+    assert O.sample_next(z, V, 0.0, 50, 0.7) == best
+    order = np.argsort(-z[:V], kind="stable")
+    assert O.sample_next(z, V, 1.0, 5, 0.0) == order[0]          # u = 0: the largest logit
+    assert O.sample_next(z, V, 1.0, 5, 1 - 1e-12) == order[4]    # u -> 1: the k-th largest
+    assert O.sample_next(z, V, 1e-6, 5, 0.999) == order[0]       # temperature -> 0: greedy
+
+
+def test_sample_next_ties_go_to_lower_id():
+    z = np.array([1.0, 3.0, 2.0, 2.0, 2.0, 0.0])
+    # top 2 = id 1 and, among the three tied at 2.0, the lowest id 2
+    draws = {O.sample_next(z, 6, 1.0, 2, u) for u in np.linspace(0, 0.999, 200)}
+    assert draws == {1, 2}
+
+
+def test_sample_next_frequencies_follow_softmax():
+    """Over u spread evenly in [0, 1) the draws land on each of the top-k ids
+    with the softmax(z / T) probability restricted to them (the inverse-CDF
+    rule), up to the 1/n grid."""
+    z = np.array([0.5, 2.0, -1.0, 1.5, 0.0, 3.0, -2.0, 1.0])
+    T, k, n = 0.7, 4, 20000
+    counts = np.zeros(len(z))
+    for u in (np.arange(n) + 0.5) / n:
+        counts[O.sample_next(z, len(z), T, k, u)] += 1
+    top = np.argsort(-z)[:k]
+    p = np.zeros(len(z))
+    p[top] = np.exp(z[top] / T) / np.exp(z[top] / T).sum()
+    np.testing.assert_allclose(counts / n, p, atol=2.0 / n)
