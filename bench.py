@@ -145,7 +145,10 @@ def run_reference(args):
     value = accum * B * T / step_s
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_seq * 1e3, "higher_is_better": True,
+        "step": f"one sampled {T}-token sequence forward+backward (the timed unit); the value extrapolates "
+                f"to the {accum * B * T}-token optimizer step, {step_s:.0f} s",
+        "ms_per_optimizer_step_extrapolated": step_s * 1e3,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (Zipf 1.1 token stream)",
         "config": workload_config(args.workload),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": NCORES, "kind": "oracle",

@@ -430,8 +430,8 @@ static_assert(DKV_STAGE_BYTES % 1024 == 0, "ring stages keep the 1024-byte swizz
 
 __global__ void __launch_bounds__(BW_THREADS, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                const float* __restrict__ ld_in, bf16* __restrict__ dqkv, float* __restrict__ colsum, int T, int H,
-                int BH, float scale, float sl2) {
+                const float* __restrict__ ld_in, bf16* __restrict__ dqkv, float* __restrict__ colsum,
+                bf16* __restrict__ ds_out, int T, int H, int BH, float scale, float sl2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
@@ -648,6 +648,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             dv[(c >> 1) + e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
           }
         }
+        if (ds_out != nullptr) {
+          // dS^T of this block for dq_mma_kernel: tile (bh, query block i,
+          // key block kb), row = key, 32 consecutive queries per warp
+          const int tile = bh * (nqb * (nqb + 1) / 2) + i * (i + 1) / 2 + kb;
+          uint32_t* dst = reinterpret_cast<uint32_t*>(ds_out + (long)tile * (BT * BT) + (kr * BT + cq * 32));
+          st32(dst, dv[0], dv[1], dv[2], dv[3], dv[4], dv[5], dv[6], dv[7]);
+          st32(dst + 8, dv[8], dv[9], dv[10], dv[11], dv[12], dv[13], dv[14], dv[15]);
+        }
         // the previous step's dV / dK MMAs have read P^T and dS^T
         if (g >= 1 && !warp_wait(p_free, (g - 1) & 1u)) {
           ok = false;
@@ -704,29 +712,263 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------- lse / D rows
+// The per-query values the backward kernels stream: lse*log2(e) and
+// D = sum_d dO[q,d] O[q,d], padded to whole 128-query blocks (+inf and 0 past
+// T), in ld[((b*H + h)*nqb + qb)*LD_FLOATS + r] and [... + BT + r].  One thread
+// per (padded row, head), heads fastest so that a warp reads contiguous rows.
+// The sum runs in the same order as in dq_kernel (four chains over pairs of
+// columns), so either route gives the same bits.
+__global__ void __launch_bounds__(256) ld_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
+                                                 const float* __restrict__ lse, float* __restrict__ ld, int B, int T,
+                                                 int H) {
+  const int nqb = (T + BT - 1) / BT;
+  const long n = (long)B * nqb * BT * H;
+  const long gi = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gi >= n) return;
+  const int h = (int)(gi % H);
+  const long m = gi / H;
+  const int b = (int)(m / ((long)nqb * BT)), q = (int)(m % ((long)nqb * BT));
+  const int C = H * HD;
+  float l2 = INFINITY, dq_ = 0.f;
+  if (q < T) {
+    l2 = lse[((long)b * H + h) * T + q] * 1.4426950408889634f;
+    const bf16* orow = out + ((long)b * T + q) * C + h * HD;
+    const bf16* drow = dout + ((long)b * T + q) * C + h * HD;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < HD / 8; ++c) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(orow + 8 * c);
+      const uint4 dv = *reinterpret_cast<const uint4*>(drow + 8 * c);
+      const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w}, d4[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 of = unpack_bf16x2(o4[e]), df = unpack_bf16x2(d4[e]);
+        acc[e] = fmaf(of.x, df.x, fmaf(of.y, df.y, acc[e]));
+      }
+    }
+    dq_ = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  }
+  float* ldb = ld + (((long)b * H + h) * nqb + q / BT) * LD_FLOATS;
+  ldb[q % BT] = l2;
+  ldb[BT + q % BT] = dq_;
+}
+
+// ----------------------------------------------------- dQ from stored dS
+// dQ_i = sum_{j <= i} dS_ij K_j / sqrt(d), with the bf16 dS tiles that
+// dkdv_kernel stored (tile (bh, i, j) holds dS^T: row = key, 128 queries), so
+// no score is formed twice.  Persistent, one CTA per SM, items (128 queries of
+// one (batch, head)) longest first.  Warp 0 streams (dS_ij, K_j) through a
+// 4-stage TMA ring; warp 1 issues dQ += dS_ij K_j (M = 128 queries, N = 64,
+// K = 128 keys, A and B both MN-major in shared memory) into one of two TMEM
+// accumulators (by item parity); warps 2..5 scale dQ, store it as bf16 and
+// form its column sums, while the next item's MMAs run.  The MMAs add the key
+// blocks in the order dq_kernel does, on the same bf16 values.
+constexpr int DQM_STAGES = 4;
+constexpr int DQM_STAGE = 3 * TILE;  // dS tile as four 64x64 boxes [key half][query half], then K_j
+constexpr int DQM_BAR_OFF = DQM_STAGES * DQM_STAGE;
+constexpr int DQM_SMEM = DQM_BAR_OFF + 256 + 1024;
+constexpr uint32_t DQM_TMEM_COLS = 128;  // two 64-column dQ accumulators
+
+__global__ void __launch_bounds__(192, 1)
+    dq_mma_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_qkv,
+                  bf16* __restrict__ dqkv, float* __restrict__ colsum, int T, int H, int BH, float scale) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQM_BAR_OFF);
+  uint64_t* full = bars;                    // DQM_STAGES
+  uint64_t* empty = full + DQM_STAGES;      // DQM_STAGES
+  uint64_t* acc_full = empty + DQM_STAGES;  // 2: the item's dQ is complete
+  uint64_t* acc_empty = acc_full + 2;       // 2, count 4: the item's dQ is in registers
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (T + BT - 1) / BT;
+  const int nitems = nqb * BH;
+  const int ntri = nqb * (nqb + 1) / 2;
+  const int C = H * HD;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DQM_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(DQM_TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_ds)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
+      uint32_t g = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+        int qb, bh;
+        item_desc(w, nqb, BH, qb, bh);
+        const int b = bh / H, h = bh % H, row0 = b * T;
+        const long trow = ((long)bh * ntri + (long)qb * (qb + 1) / 2) * BT;  // first row of tile (bh, qb, 0)
+        for (int kb = 0; kb <= qb; ++kb, ++g) {
+          const int s = g % DQM_STAGES;
+          if (!mbar_wait(&empty[s], ((g / DQM_STAGES) & 1u) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], DQM_STAGE);
+          const uint32_t dst = smem_u32(smem + s * DQM_STAGE);
+          const int y = (int)(trow + (long)kb * BT);
+          tma_load_2d(dst, &tm_ds, 0, y, &full[s]);
+          tma_load_2d(dst + 8192, &tm_ds, 64, y, &full[s]);
+          tma_load_2d(dst + 16384, &tm_ds, 0, y + 64, &full[s]);
+          tma_load_2d(dst + 24576, &tm_ds, 64, y + 64, &full[s]);
+          tma_load_2d(dst + 2 * TILE, &tm_qkv, C + h * HD, row0 + kb * BT, &full[s]);
+        }
+      }
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      drain_ring(full, DQM_STAGES, g);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = att_idesc(HD, 1) | (1u << 15);  // N = 64, A and B MN-major
+      uint32_t g = 0, t = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+        int qb, bh;
+        item_desc(w, nqb, BH, qb, bh);
+        const uint32_t ab = t & 1u;
+        if (!mbar_wait(&acc_empty[ab], ((t >> 1) & 1u) ^ 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb <= qb; ++kb, ++g) {
+          const int s = g % DQM_STAGES;
+          if (!mbar_wait(&full[s], (g / DQM_STAGES) & 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * DQM_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < BT / 16; ++kk)
+            tc_mma(tmem + ab * HD, make_sdesc(base + (kk >> 2) * 16384 + (kk & 3) * 2048, 1),
+                   make_sdesc(base + 2 * TILE + kk * 2048, 1), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+          if (kb == qb) tc_commit(&acc_full[ab]);
+        }
+      }
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      tc_commit(drain);
+      if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
+    }
+  } else {
+    // ------------------------------------------------------- epilogue
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+    uint32_t t = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < nitems; w += gridDim.x, ++t) {
+      int qb, bh;
+      item_desc(w, nqb, BH, qb, bh);
+      const int b = bh / H, h = bh % H, row0 = b * T;
+      const int q = qb * BT + r;
+      const uint32_t ab = t & 1u;
+      if (!warp_wait(&acc_full[ab], (t >> 1) & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t a0[32], a1[32];
+      tmem_ld32(tl + ab * HD, a0);
+      tmem_ld32(tl + ab * HD + 32, a1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (q < T) {
+        bf16* dst = dqkv + ((long)row0 + q) * (3L * C) + h * HD;
+        store_row32(dst, a0, scale);
+        store_row32(dst + 32, a1, scale);
+      }
+      if (colsum) {
+        const long prow = (((long)b * nqb + qb) * 4 + qw) * (3L * C) + h * HD;
+        float cs[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cs[i] = q < T ? __uint_as_float(a0[i]) * scale : 0.f;
+        const float t0 = warp_colsum32(cs, lane);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cs[i] = q < T ? __uint_as_float(a1[i]) * scale : 0.f;
+        const float t1 = warp_colsum32(cs, lane);
+        colsum[prow + lane] = t0;
+        colsum[prow + 32 + lane] = t1;
+      }
+    }
+    if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(DQM_TMEM_COLS) : "memory");
+  }
+}
+
 // fp32 scratch of the backward: lse*log2(e) and D per query, padded to whole
 // 128-query blocks
 static inline long backward_scratch_floats(int B, int T, int H) {
   return (long)B * H * ((T + BT - 1) / BT) * LD_FLOATS;
 }
+// bf16 elements of the stored dS tiles: 128 x 128 per (batch, head, query
+// block, key block at or below it)
+static inline long backward_ds_elems(int B, int T, int H) {
+  const long nqb = (T + BT - 1) / BT;
+  return (long)B * H * (nqb * (nqb + 1) / 2) * BT * BT;
+}
 // rows of the column-sum partials: one per (batch, 128-row block, lane quarter)
 static inline long backward_colsum_rows(int B, int T) { return (long)B * ((T + BT - 1) / BT) * 4; }
 
-// dq_kernel first (it also writes lse*log2(e) and D into `ld`), then
-// dkdv_kernel.  ld: fp32 scratch of backward_scratch_floats(B, T, H) elements,
-// 16-byte aligned.  colsum (may be null): [backward_colsum_rows(B, T)][3C]
-// fp32 partial column sums of dqkv (summing them over the rows gives the qkv
-// bias gradient).
+// The attention backward.  ld: fp32 scratch of backward_scratch_floats(B, T,
+// H) elements, 16-byte aligned.  colsum (may be null): [backward_colsum_rows(B,
+// T)][3C] fp32 partial column sums of dqkv (summing them over the rows gives
+// the qkv bias gradient).
+//  ds given (backward_ds_elems(B, T, H) bf16, 16-byte aligned): ld_kernel forms
+//     lse*log2(e) and D, dkdv_kernel forms P and dS once per score and stores
+//     dS, dq_mma_kernel reads it back for dQ (three launches).
+//  ds null: dq_kernel forms D and dQ from recomputed scores, then dkdv_kernel
+//     (two launches, no scratch beyond ld).
+// Both routes run the same arithmetic on every score (the products of S and
+// dP are the same bf16 pairs in either operand order, and every sum runs in
+// the same order), so their results agree bit for bit.
 static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, bf16* dqkv,
-                                   float* ld, int B, int T, int H, cudaStream_t st, float* colsum = nullptr) {
+                                   float* ld, int B, int T, int H, cudaStream_t st, float* colsum = nullptr,
+                                   bf16* ds = nullptr) {
   static DeviceOnce once;
   cudaError_t e = run_once_per_device(once, [] {
     cudaError_t r = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM);
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(dq_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQM_SMEM);
     return r;
   });
   if (e != cudaSuccess) return e;
-  if (reinterpret_cast<uintptr_t>(ld) & 15) return cudaErrorInvalidValue;
+  if ((reinterpret_cast<uintptr_t>(ld) & 15) || (reinterpret_cast<uintptr_t>(ds) & 15)) return cudaErrorInvalidValue;
   const int C = H * HD;
   CUtensorMap tq, td;
   if (make_tmap(&tq, qkv, 3L * C, (long)B * T, 3L * C, 64, BT) != 0) return cudaErrorInvalidValue;
@@ -735,8 +977,17 @@ static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16*
   const float sl2 = 1.4426950408889634f * scale;
   const int items = ((T + BT - 1) / BT) * B * H;
   const int grid = items < num_sms_attn() ? items : num_sms_attn();
-  dq_kernel<<<grid, BW_THREADS, DQ_SMEM, st>>>(tq, td, out, lse, ld, dqkv, colsum, T, H, B * H, scale, sl2);
-  dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, T, H, B * H, scale, sl2);
+  if (ds != nullptr) {
+    CUtensorMap tds;
+    if (make_tmap(&tds, ds, BT, backward_ds_elems(B, T, H) / BT, BT, 64, 64) != 0) return cudaErrorInvalidValue;
+    const long n = (long)B * ((T + BT - 1) / BT) * BT * H;
+    ld_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
+    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, ds, T, H, B * H, scale, sl2);
+    dq_mma_kernel<<<grid, 192, DQM_SMEM, st>>>(tds, tq, dqkv, colsum, T, H, B * H, scale);
+  } else {
+    dq_kernel<<<grid, BW_THREADS, DQ_SMEM, st>>>(tq, td, out, lse, ld, dqkv, colsum, T, H, B * H, scale, sl2);
+    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, nullptr, T, H, B * H, scale, sl2);
+  }
   return cudaGetLastError();
 }
 

@@ -332,30 +332,54 @@ __global__ void __launch_bounds__(LN_BWD_WARPS * 32, 2) ln_bwd_kernel(const TI* 
 }
 
 // Sum per-block partial rows (fixed order) into up to three outputs:
-// part is [nblk][ncols]; column j goes to out[j / C][j % C] (+=).  One warp
-// per 32 columns and block; the 8 warps of a block take every 8th partial row
-// and are combined in warp order, so the result is independent of timing.
-__global__ void __launch_bounds__(256) partials_reduce_kernel(const float* __restrict__ part, int nblk, int ncols, int C,
-                                                              float* __restrict__ out0, float* __restrict__ out1,
-                                                              float* __restrict__ out2) {
+// part is [nblk][ncols]; column j goes to out[j / C][j % C] (+=).  A cluster
+// of PR_SPLIT CTAs serves 32 columns: warp w of CTA y sums the partial rows
+// b = 8y + w (mod 8*PR_SPLIT) in ascending order, each CTA combines its warps
+// in warp order, and CTA 0 adds the CTAs' sums in rank order through
+// distributed shared memory, so the result is independent of timing.
+constexpr int PR_SPLIT = 8;
+__global__ void __cluster_dims__(1, PR_SPLIT, 1) __launch_bounds__(256)
+    partials_reduce_kernel(const float* __restrict__ part, int nblk, int ncols, int C, float* __restrict__ out0,
+                           float* __restrict__ out1, float* __restrict__ out2) {
   __shared__ float red[8][32];
+  __shared__ float tot[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
+  uint32_t rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
   float s = 0.f;
   if (col < ncols) {
-#pragma unroll 8
-    for (int b = warp; b < nblk; b += 8) s += part[(long)b * ncols + col];
+#pragma unroll 4
+    for (int b = 8 * (int)rank + warp; b < nblk; b += 8 * PR_SPLIT) s += part[(long)b * ncols + col];
   }
   red[warp][lane] = s;
   __syncthreads();
-  if (warp == 0 && col < ncols) {
+  if (warp == 0) {
     float t = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) t += red[w][lane];
-    const int which = col / C, c = col % C;
-    float* o = which == 0 ? out0 : (which == 1 ? out1 : out2);
-    if (o != nullptr) o[c] += t;
+    tot[lane] = t;
   }
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (rank == 0 && warp == 0) {
+    const uint32_t local = (uint32_t)__cvta_generic_to_shared(&tot[lane]);
+    float t = 0.f;
+#pragma unroll
+    for (uint32_t r = 0; r < PR_SPLIT; ++r) {
+      uint32_t remote;
+      float v;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(r));
+      asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+      t += v;
+    }
+    if (col < ncols) {
+      const int which = col / C, c = col % C;
+      float* o = which == 0 ? out0 : (which == 1 ? out1 : out2);
+      if (o != nullptr) o[c] += t;
+    }
+  }
+  // no CTA leaves while CTA 0 may still read its shared memory
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Column sums of an [M, N] matrix, stage 1: block (x, y) sums 32 column

@@ -314,7 +314,8 @@ int gpt2_attention_forward(const void* qkv, void* out, float* lse, int B, int T,
 
 int64_t gpt2_attention_workspace_floats(int B, int T, int H) {
   if (B < 1 || T < 1 || H < 1) return 0;
-  return (int64_t)tcfa::backward_scratch_floats(B, T, H);
+  // lse*log2(e) and D rows, then the bf16 dS tiles (1 KB aligned)
+  return (int64_t)tcfa::backward_scratch_floats(B, T, H) + (tcfa::backward_ds_elems(B, T, H) + 1) / 2;
 }
 
 int gpt2_attention_backward(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv,
@@ -322,8 +323,9 @@ int gpt2_attention_backward(const void* qkv, const void* out, const void* dout, 
   if (!qkv || !out || !dout || !lse || !dqkv || !work || !attn_sizes_ok(B, T, H)) return GPT2_EINVAL;
   if (!aligned16(qkv) || !aligned16(out) || !aligned16(dout) || !aligned16(dqkv) || !aligned16(work))
     return GPT2_EINVAL;
+  bf16* ds = reinterpret_cast<bf16*>(work + tcfa::backward_scratch_floats(B, T, H));
   return tcfa::backward((const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, (bf16*)dqkv, work, B, T, H,
-                              (cudaStream_t)stream) == cudaSuccess
+                        (cudaStream_t)stream, nullptr, ds) == cudaSuccess
              ? GPT2_OK
              : GPT2_ECUDA;
 }

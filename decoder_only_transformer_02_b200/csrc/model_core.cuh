@@ -52,6 +52,7 @@ struct gpt2 {
   float *ce_lse = nullptr, *losses = nullptr, *d_loss = nullptr;
   float* ce_part = nullptr;  // lm_head softmax statistics per (row, 128 columns) (bf16 mode)
   float* attn_cs = nullptr;  // per-128-row-block column sums of dqkv from the attention backward (bf16 mode)
+  bf16* attn_ds = nullptr;   // the attention backward's dS tiles, one layer at a time (bf16 mode)
   int32_t* argmax = nullptr;
 
   // backward scratch
@@ -214,7 +215,7 @@ static void free_all(gpt2* h) {
                   h->ce_lse,  h->losses,  h->d_loss,   h->argmax,   h->dres,     h->dln,      h->attn_D,
                   h->ln_part, h->cs_part, h->dres_bf,  h->dbig,     h->dqkv,     h->datt,     h->splitk_ws,
                   h->emb_keys, h->emb_part, h->normbuf, h->d_step, h->norm_part, h->segs,    h->d_bad,    h->tok_dev,
-                  h->tgt_dev, h->ce_part, h->attn_cs, h->kv, h->dec_x, h->dec_mean, h->dec_rstd, h->dec_ln,
+                  h->tgt_dev, h->ce_part, h->attn_cs, h->attn_ds, h->kv, h->dec_x, h->dec_mean, h->dec_rstd, h->dec_ln,
                   h->dec_qkv, h->dec_att, h->dec_u, h->dec_a, h->dec_logits};
   for (void* p : ptrs)
     if (p) cudaFree(p);

@@ -115,6 +115,7 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   if (h->prec == GPT2_BF16) {
     ALLOC(h, h->ce_part, (size_t)Mx * tcg::ce_halves(h->Vp) * 3 * 4);
     ALLOC(h, h->attn_cs, (size_t)tcfa::backward_colsum_rows(h->maxB, h->maxT) * 3 * C * 4);
+    ALLOC(h, h->attn_ds, (size_t)tcfa::backward_ds_elems(h->maxB, h->maxT, H) * 2);
   }
   ALLOC(h, h->losses, (size_t)Mx * 4);
   ALLOC(h, h->d_loss, 16);

@@ -52,7 +52,7 @@ static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean
       return set_err(h, GPT2_EINVAL, "n_embd must be a multiple of 128 up to 1024");
   }
   LAUNCH_CHECK(h);
-  k::partials_reduce_kernel<<<(3 * h->C + 31) / 32, 256, 0, h->stream>>>(
+  k::partials_reduce_kernel<<<dim3((3 * h->C + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(
       h->ln_part, nblk, 3 * h->C, h->C, h->G32(goff), h->G32(boff),
       dbias_off == NO_OFF ? nullptr : h->G32(dbias_off));
   LAUNCH_CHECK(h);
@@ -232,7 +232,7 @@ static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
   else
     k::colsum_partial_kernel<float><<<grid, 256, 0, h->stream>>>((const float*)a, (int)M, N, rpb, h->cs_part);
   LAUNCH_CHECK(h);
-  k::partials_reduce_kernel<<<(N + 31) / 32, 256, 0, h->stream>>>(h->cs_part, nblk, N, N, h->G32(boff), nullptr,
+  k::partials_reduce_kernel<<<dim3((N + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(h->cs_part, nblk, N, N, h->G32(boff), nullptr,
                                                                    nullptr);
   LAUNCH_CHECK(h);
   return GPT2_OK;
@@ -243,7 +243,7 @@ static int op_attn_bias_reduce(gpt2* h, size_t boff) {
   KTimer kt(h, KC_OTHER, 0.0, 0.0);
   const int nblk = (int)tcfa::backward_colsum_rows(h->B, h->T);
   const int n = 3 * h->C;
-  k::partials_reduce_kernel<<<(n + 31) / 32, 256, 0, h->stream>>>(h->attn_cs, nblk, n, n, h->G32(boff), nullptr,
+  k::partials_reduce_kernel<<<dim3((n + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(h->attn_cs, nblk, n, n, h->G32(boff), nullptr,
                                                                   nullptr);
   LAUNCH_CHECK(h);
   return GPT2_OK;
@@ -277,9 +277,9 @@ static int op_attn_bwd(gpt2* h, int l) {
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;
   if (h->prec == GPT2_BF16) {
     if (tcfa::backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
-                       h->B, h->T, h->H, h->stream, h->attn_cs) != cudaSuccess)
+                       h->B, h->T, h->H, h->stream, h->attn_cs, h->attn_ds) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention backward launch");
-    h->launches += 2;
+    h->launches += 3;
   } else {
     if (attn::naive_backward((const float*)qkv, (const float*)att, (const float*)h->datt, lse, (float*)h->dqkv,
                              h->attn_D, h->B, h->T, h->H, h->C / h->H, h->stream) != cudaSuccess)

@@ -204,10 +204,13 @@ const char* gpt2_last_error(const gpt2_t* h);
 int gpt2_attention_forward(const void* d_qkv, void* d_out, float* d_lse, int B, int T, int H, void* cuda_stream);
 /* Backward of gpt2_attention_forward: d_dqkv [B, T, 3C] bf16 receives dq, dk,
  * dv in the same column layout.  d_work: caller-provided fp32 scratch of at
- * least gpt2_attention_workspace_floats(B, T, H) elements, 16-byte aligned
- * (lse*log2(e) and D = rowsum(dO * O) for every query, in whole blocks of 128
- * queries: 2*B*H*ceil(T/128)*128 floats).  Deterministic: the same inputs
- * give the same bits. */
+ * least gpt2_attention_workspace_floats(B, T, H) elements, 16-byte aligned:
+ * lse*log2(e) and D = rowsum(dO * O) for every query, in whole blocks of 128
+ * queries (2*B*H*ceil(T/128)*128 floats), then the bf16 dS = P * (dP - D)
+ * tiles of 128 x 128 for every (batch, head, query block, key block at or
+ * below it) (B*H*n*(n+1)/2 tiles, n = ceil(T/128), 32 KB each).  dS is formed
+ * once per score by the dK/dV kernel and read back for dQ.  Deterministic:
+ * the same inputs give the same bits. */
 int gpt2_attention_backward(const void* d_qkv, const void* d_out, const void* d_dout, const float* d_lse,
                             void* d_dqkv, float* d_work, int B, int T, int H, void* cuda_stream);
 int64_t gpt2_attention_workspace_floats(int B, int T, int H);
@@ -258,7 +261,9 @@ int gpt2_set_wait_limit_ns(uint64_t limit_ns);
  * (batch, head, position) row, rows padded to whole blocks of 128 positions)
  * lives in a fixed array inside the library of 2 * GPT2_ATTN_NOALLOC_MAX_ROWS
  * floats (4 MiB); every GPU that loads the library holds that array until the
- * process exits.
+ * process exits.  Having no room for the dS tiles, it forms dQ from scores
+ * recomputed in a dQ kernel of its own instead of reading dS back; that kernel
+ * does the same arithmetic on every score in the same order.
  *  - B*H*ceil(T/128)*128 must be at most GPT2_ATTN_NOALLOC_MAX_ROWS and B*H at
  *    most 65535, else GPT2_EINVAL and nothing is enqueued.  Other arguments as
  *    for gpt2_attention_backward, whose results it reproduces bit for bit.
