@@ -100,15 +100,18 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle
 
+SAMPLE_B = 2  # sequences per timed oracle sample (about 15 s of host time at T=1024)
+
+
 def oracle_sample(T: int, seed: int):
-    """The oracle as it stands, fp32, on one sequence of the workload: forward +
-    backward of B=1 x T tokens, and one AdamW update over all parameters.
-    Returns (seconds for fwd+bwd of one sequence, seconds for AdamW)."""
+    """The oracle as it stands, fp32, on a slice of one micro-step of the
+    workload: forward + backward of SAMPLE_B x T tokens, and one AdamW update
+    over all parameters.  Returns (seconds for the fwd+bwd, seconds for AdamW)."""
     from decoder_only_transformer_02_b200 import synthetic as S
     from oracle import gpt2_oracle as O
     cfg = O.GPT2_124M
     flat = O.init_params(cfg, 1234, dtype=np.float32)
-    (tok, tgt), = S.token_batches("zipf", V, 1, T, 1, seed=seed)
+    (tok, tgt), = S.token_batches("zipf", V, SAMPLE_B, T, 1, seed=seed)
     t0 = time.perf_counter()
     st = O.forward(flat, cfg, tok, tgt)
     g = O.backward(st, 1.0)
@@ -119,10 +122,10 @@ def oracle_sample(T: int, seed: int):
 
 
 def cpu_baseline(B, T, accum, seed=7):
-    t_seq, t_adam = oracle_sample(T, seed)
-    step_s = accum * B * t_seq + t_adam
+    t_smp, t_adam = oracle_sample(T, seed)
+    step_s = accum * B / SAMPLE_B * t_smp + t_adam
     return {"value": accum * B * T / step_s, "unit": "tokens/s", "cores": NCORES, "kind": "oracle",
-            "sample": f"one {T}-token sequence forward+backward ({t_seq:.2f} s) and one AdamW update over "
+            "sample": f"forward+backward of {SAMPLE_B} x {T} tokens ({t_smp:.2f} s) and one AdamW update over "
                       f"{N_PARAMS} params ({t_adam:.2f} s), NumPy fp32; optimizer step = {accum * B} sequences "
                       f"+ 1 update, extrapolated"}
 
@@ -140,20 +143,21 @@ def run_reference(args):
     times = []
     for k in range(args.steps):
         times.append(oracle_sample_fwd_bwd(T, 200 + k))
-    t_seq = sum(times) / len(times)
-    step_s = accum * B * t_seq + t_adam
+    t_smp = sum(times) / len(times)
+    step_s = accum * B / SAMPLE_B * t_smp + t_adam
     value = accum * B * T / step_s
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_seq * 1e3, "higher_is_better": True,
-        "step": f"one sampled {T}-token sequence forward+backward (the timed unit); the value extrapolates "
-                f"to the {accum * B * T}-token optimizer step, {step_s:.0f} s",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_smp * 1e3, "higher_is_better": True,
+        "step": f"one sampled forward+backward of {SAMPLE_B} x {T} tokens (the timed unit); the value "
+                f"extrapolates to the {accum * B * T}-token optimizer step, {step_s:.0f} s",
         "ms_per_optimizer_step_extrapolated": step_s * 1e3,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (Zipf 1.1 token stream)",
         "config": workload_config(args.workload),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": NCORES, "kind": "oracle",
-                         "sample": f"each step: one {T}-token sequence forward+backward of the NumPy fp32 oracle "
-                                   f"(mean {t_seq:.2f} s); AdamW over all params measured once ({t_adam:.2f} s); "
+                         "sample": f"each step: forward+backward of {SAMPLE_B} x {T} tokens by the NumPy fp32 "
+                                   f"oracle (mean {t_smp:.2f} s); AdamW over all params measured once "
+                                   f"({t_adam:.2f} s); "
                                    f"optimizer step = {accum * B} sequences + 1 update, extrapolated"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -168,7 +172,7 @@ def oracle_sample_fwd_bwd(T, seed):
     global _ORACLE_FLAT
     if "_ORACLE_FLAT" not in globals():
         _ORACLE_FLAT = O.init_params(cfg, 1234, dtype=np.float32)
-    (tok, tgt), = S.token_batches("zipf", V, 1, T, 1, seed=seed)
+    (tok, tgt), = S.token_batches("zipf", V, SAMPLE_B, T, 1, seed=seed)
     t0 = time.perf_counter()
     st = O.forward(_ORACLE_FLAT, cfg, tok, tgt)
     O.backward(st, 1.0)

@@ -143,6 +143,15 @@ constexpr float RESCALE_LOG2 = 8.f;                       // lazy-rescale thresh
 #define EX2_FMA_EVERY 0  // > 0: one pair of exponentials in EX2_FMA_EVERY through ex2_fma instead of MUFU
 #endif
 
+// The k-th work item of this CTA: items are numbered longest first and dealt
+// to the CTAs in a snake order (CTA c takes c, 2G-1-c, 2G+c, 4G-1-c, ... for a
+// grid of G), so each CTA's long and short items balance out; the sequence
+// increases in k.
+__device__ __forceinline__ int snake_item(int k) {
+  const int G = gridDim.x, c = blockIdx.x;
+  return k * G + ((k & 1) ? G - 1 - c : c);
+}
+
 // The w-th work item in descending order of length: 128-row block index and
 // (batch, head) row of the grid.
 __device__ __forceinline__ void item_desc(int w, int nblk, int BH, int& blk, int& bh) {
@@ -205,7 +214,7 @@ __global__ void __launch_bounds__(192, 2)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
       uint32_t g = 0, t = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int qb, bh;
         item_desc(w, nqb, BH, qb, bh);
         const int b = bh / H, h = bh % H, row0 = b * T;
@@ -265,7 +274,7 @@ __global__ void __launch_bounds__(192, 2)
         tc_commit(pv_done);
         return true;
       };
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int qb, bh;
         item_desc(w, nqb, BH, qb, bh);
         const int nkv = min(qb * BQ + BQ - 1, T - 1) / BKV + 1;
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t g = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+    for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k)) {
       int qb, bh;
       item_desc(w, nqb, BH, qb, bh);
       const int b = bh / H, h = bh % H;

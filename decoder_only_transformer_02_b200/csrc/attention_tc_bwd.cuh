@@ -112,6 +112,19 @@ __device__ __forceinline__ void drain_ring(uint64_t* bars, int n, uint32_t issue
   }
 }
 
+// TMA tile store shared -> global (bulk-group completion) and its waits
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the committed stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the committed stores are complete
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ----------------------------------------------------------------- dQ
 // Shared memory: two buffers of (Q, dO) 128x64 tiles (16 KB each, 128-byte
 // swizzled K-major rows of 64 bf16), then the ring of K_j, V_j tiles.
@@ -187,7 +200,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_do)) : "memory");
       uint32_t g = 0, t = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int qb, bh;
         item_desc(w, nqb, BH, qb, bh);
         const int b = bh / H, h = bh % H, row0 = b * T;
@@ -241,7 +254,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         if (last) tc_commit(&acc_full[ab]);
         return true;
       };
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int qb, bh;
         item_desc(w, nqb, BH, qb, bh);
         const int nblk = min(qb * BT + BT - 1, T - 1) / BT + 1;
@@ -291,7 +304,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     float* Dsm = reinterpret_cast<float*>(smem + DQ_D_OFF);  // [item parity][lse2 128, D 128]
     uint32_t g = 0, t = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+    for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
       int qb, bh;
       item_desc(w, nqb, BH, qb, bh);
       const int b = bh / H, h = bh % H, row0 = b * T;
@@ -417,11 +430,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
 
 // ------------------------------------------------------------ dK, dV
 // Shared memory: two buffers of (K, V) 128x64 tiles, then the ring of Q_i,
-// dO_i tiles and the block's lse*log2(e) / D rows (33 KB per stage).
+// dO_i tiles and the block's lse*log2(e) / D rows (33 KB per stage), then the
+// staging tile of dS^T for its TMA store (four 64x64 boxes, [key half][query
+// half], 128-byte swizzled rows).
+constexpr int DKV_STAGES = 3;
 constexpr int DKV_KV_OFF = 0;                              // buffer b: K at +2b*TILE, V at +(2b+1)*TILE
 constexpr int DKV_STAGE_BYTES = 2 * TILE + LD_FLOATS * 4;
 constexpr int DKV_RING_OFF = 4 * TILE;                     // stage s: Q, dO, lse2/D
-constexpr int DKV_BAR_OFF = DKV_RING_OFF + BW_STAGES * DKV_STAGE_BYTES;
+constexpr int DKV_DS_OFF = DKV_RING_OFF + DKV_STAGES * DKV_STAGE_BYTES;
+constexpr int DKV_BAR_OFF = DKV_DS_OFF + 2 * TILE;
 constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
 // P^T (bf16 pairs) [384,448), dS^T (bf16 pairs) [448,512)
@@ -430,22 +447,24 @@ static_assert(DKV_STAGE_BYTES % 1024 == 0, "ring stages keep the 1024-byte swizz
 
 __global__ void __launch_bounds__(BW_THREADS, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                const float* __restrict__ ld_in, bf16* __restrict__ dqkv, float* __restrict__ colsum,
-                bf16* __restrict__ ds_out, int T, int H, int BH, float scale, float sl2) {
+                const __grid_constant__ CUtensorMap tm_ds, const float* __restrict__ ld_in, bf16* __restrict__ dqkv,
+                float* __restrict__ colsum, int store_ds, int T, int H, int BH, float scale, float sl2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DKV_BAR_OFF);
   uint64_t* kv_full = bars;                  // 2: K and V tiles
   uint64_t* kv_empty = bars + 2;             // 2: the item's last S^T / dP^T MMA has read them
-  uint64_t* qd_full = bars + 4;              // BW_STAGES
-  uint64_t* qd_empty = qd_full + BW_STAGES;  // BW_STAGES
-  uint64_t* s_full = qd_empty + BW_STAGES;   // S^T and dP^T in TMEM
+  uint64_t* qd_full = bars + 4;              // DKV_STAGES
+  uint64_t* qd_empty = qd_full + DKV_STAGES;  // DKV_STAGES
+  uint64_t* s_full = qd_empty + DKV_STAGES;   // S^T and dP^T in TMEM
   uint64_t* s_free = s_full + 1;             // count BW_CWARPS
   uint64_t* p_full = s_free + 1;             // count BW_CWARPS: P^T and dS^T in TMEM
   uint64_t* p_free = p_full + 1;             // the dV / dK MMAs have read them
   uint64_t* acc_done = p_free + 1;           // the item's dV / dK are complete
   uint64_t* drain = acc_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* st_full = drain + 1;             // count BW_CWARPS: the dS^T staging tile is written
+  uint64_t* st_free = st_full + 1;           // the previous tile's TMA store has read the staging tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(st_free + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (T + BT - 1) / BT;
@@ -457,7 +476,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int s = 0; s < BW_STAGES; ++s) {
+    for (int s = 0; s < DKV_STAGES; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
     }
@@ -467,6 +486,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     mbar_init(p_free, 1);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
+    mbar_init(st_full, BW_CWARPS);
+    mbar_init(st_free, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -493,7 +514,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_do)) : "memory");
       uint32_t g = 0, t = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int kb, bh;
         item(w, kb, bh);
         const int b = bh / H, h = bh % H, row0 = b * T;
@@ -508,8 +529,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         tma_load_2d(kd, &tm_qkv, C + h * HD, row0 + kb * BT, &kv_full[kvb]);
         tma_load_2d(kd + TILE, &tm_qkv, 2 * C + h * HD, row0 + kb * BT, &kv_full[kvb]);
         for (int n = 0; n < nblk; ++n, ++g) {
-          const int i = kb + n, s = g % BW_STAGES;
-          if (!mbar_wait(&qd_empty[s], ((g / BW_STAGES) & 1u) ^ 1u)) {
+          const int i = kb + n, s = g % DKV_STAGES;
+          if (!mbar_wait(&qd_empty[s], ((g / DKV_STAGES) & 1u) ^ 1u)) {
             ok = false;
             break;
           }
@@ -521,7 +542,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
       }
       if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
-      drain_ring(qd_full, BW_STAGES, g);
+      drain_ring(qd_full, DKV_STAGES, g);
       drain_ring(kv_full, 2, t);
     }
   } else if (warp == 1) {
@@ -535,7 +556,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       auto acc_step = [&](uint32_t gp, int np, int last) -> bool {
         if (!mbar_wait(p_full, gp & 1u)) return false;
         tc_fence_after();
-        const int s = gp % BW_STAGES;
+        const int s = gp % DKV_STAGES;
         const uint32_t qa = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
         const uint32_t doa = qa + TILE;
 #pragma unroll
@@ -549,7 +570,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         if (last) tc_commit(acc_done);
         return true;
       };
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int kb, bh;
         item(w, kb, bh);
         const int nblk = nqb - kb;
@@ -560,8 +581,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
         const uint32_t ka = smem_u32(smem + DKV_KV_OFF + 2 * kvb * TILE), va = ka + TILE;
         for (int n = 0; n < nblk; ++n, ++g) {
-          const int s = g % BW_STAGES;
-          if (!mbar_wait(&qd_full[s], (g / BW_STAGES) & 1u) || (g >= 1 && !mbar_wait(s_free, (g - 1) & 1u))) {
+          const int s = g % DKV_STAGES;
+          if (!mbar_wait(&qd_full[s], (g / DKV_STAGES) & 1u) || (g >= 1 && !mbar_wait(s_free, (g - 1) & 1u))) {
             ok = false;
             break;
           }
@@ -597,15 +618,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t g = 0, t = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+    for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
       int kb, bh;
       item(w, kb, bh);
       const int b = bh / H, h = bh % H, row0 = b * T;
       const int nblk = nqb - kb;
       const int key = kb * BT + kr;  // key position
       for (int n = 0; n < nblk; ++n, ++g) {
-        const int i = kb + n, s = g % BW_STAGES;
-        if (!warp_wait(s_full, g & 1u) || !warp_wait(&qd_full[s], (g / BW_STAGES) & 1u)) {
+        const int i = kb + n, s = g % DKV_STAGES;
+        if (!warp_wait(s_full, g & 1u) || !warp_wait(&qd_full[s], (g / DKV_STAGES) & 1u)) {
           ok = false;
           break;
         }
@@ -648,13 +669,41 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             dv[(c >> 1) + e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
           }
         }
-        if (ds_out != nullptr) {
-          // dS^T of this block for dq_mma_kernel: tile (bh, query block i,
-          // key block kb), row = key, 32 consecutive queries per warp
-          const int tile = bh * (nqb * (nqb + 1) / 2) + i * (i + 1) / 2 + kb;
-          uint32_t* dst = reinterpret_cast<uint32_t*>(ds_out + (long)tile * (BT * BT) + (kr * BT + cq * 32));
-          st32(dst, dv[0], dv[1], dv[2], dv[3], dv[4], dv[5], dv[6], dv[7]);
-          st32(dst + 8, dv[8], dv[9], dv[10], dv[11], dv[12], dv[13], dv[14], dv[15]);
+        if (store_ds) {
+          // dS^T of this block for dq_mma_kernel, tile (bh, query block i,
+          // key block kb): written into the swizzled staging tile, then one
+          // thread stores it with TMA.  The staging tile is reused once the
+          // previous tile's store has read it.
+          const bool elected = warp == 2 && lane == 0;
+          if (elected && g >= 1) {
+            bulk_wait_read0();
+            mbar_arrive(st_free);
+          }
+          if (!warp_wait(st_free, (g & 1u) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          const int rb = (qw & 1) * 32 + lane;  // row within its 64-row box
+          uint8_t* box = smem + DKV_DS_OFF + ((qw >> 1) * 2 + (cq >> 1)) * 8192;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(box + sw128(rb, (cq & 1) * 4 + c4)) =
+                make_uint4(dv[4 * c4], dv[4 * c4 + 1], dv[4 * c4 + 2], dv[4 * c4 + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(st_full);
+          if (elected) {
+            if (!mbar_wait(st_full, g & 1u)) {
+              set_device_err(DERR_WAIT_TIMEOUT);
+            } else {
+              const int y = (bh * (nqb * (nqb + 1) / 2) + i * (i + 1) / 2 + kb) * BT;
+#pragma unroll
+              for (int bx = 0; bx < 4; ++bx)
+                tma_store_2d(&tm_ds, (bx & 1) * 64, y + (bx >> 1) * 64, smem_u32(smem + DKV_DS_OFF + bx * 8192));
+              bulk_commit();
+            }
+          }
+          __syncwarp();
         }
         // the previous step's dV / dK MMAs have read P^T and dS^T
         if (g >= 1 && !warp_wait(p_free, (g - 1) & 1u)) {
@@ -704,6 +753,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       }
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+    if (warp == 2 && lane == 0) bulk_wait0();  // the dS^T stores are complete before the CTA exits
   }
   __syncthreads();
   if (warp == 1) {
@@ -718,7 +768,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
 // T), in ld[((b*H + h)*nqb + qb)*LD_FLOATS + r] and [... + BT + r].  One thread
 // per (padded row, head), heads fastest so that a warp reads contiguous rows.
 // The sum runs in the same order as in dq_kernel (four chains over pairs of
-// columns), so either route gives the same bits.
+// columns), so either route gives the same bits.  V32: out and dout are
+// 32-byte aligned (rows are read as 32-byte vectors), else 16-byte vectors.
+template <bool V32>
 __global__ void __launch_bounds__(256) ld_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
                                                  const float* __restrict__ lse, float* __restrict__ ld, int B, int T,
                                                  int H) {
@@ -735,15 +787,29 @@ __global__ void __launch_bounds__(256) ld_kernel(const bf16* __restrict__ out, c
     l2 = lse[((long)b * H + h) * T + q] * 1.4426950408889634f;
     const bf16* orow = out + ((long)b * T + q) * C + h * HD;
     const bf16* drow = dout + ((long)b * T + q) * C + h * HD;
+    // the whole 128-byte rows in flight at once
+    uint32_t ov[HD / 16][8], dv[HD / 16][8];
+#pragma unroll
+    for (int c = 0; c < HD / 16; ++c) {
+      if constexpr (V32) {
+        ld32(orow + 16 * c, ov[c]);
+        ld32(drow + 16 * c, dv[c]);
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint4 o = *reinterpret_cast<const uint4*>(orow + 16 * c + 8 * hh);
+          const uint4 d = *reinterpret_cast<const uint4*>(drow + 16 * c + 8 * hh);
+          ov[c][4 * hh] = o.x, ov[c][4 * hh + 1] = o.y, ov[c][4 * hh + 2] = o.z, ov[c][4 * hh + 3] = o.w;
+          dv[c][4 * hh] = d.x, dv[c][4 * hh + 1] = d.y, dv[c][4 * hh + 2] = d.z, dv[c][4 * hh + 3] = d.w;
+        }
+      }
+    }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < HD / 8; ++c) {
-      const uint4 ov = *reinterpret_cast<const uint4*>(orow + 8 * c);
-      const uint4 dv = *reinterpret_cast<const uint4*>(drow + 8 * c);
-      const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w}, d4[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 of = unpack_bf16x2(o4[e]), df = unpack_bf16x2(d4[e]);
+        const float2 of = unpack_bf16x2(ov[c / 2][4 * (c % 2) + e]), df = unpack_bf16x2(dv[c / 2][4 * (c % 2) + e]);
         acc[e] = fmaf(of.x, df.x, fmaf(of.y, df.y, acc[e]));
       }
     }
@@ -819,7 +885,7 @@ __global__ void __launch_bounds__(192, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_qkv)) : "memory");
       uint32_t g = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k)) {
         int qb, bh;
         item_desc(w, nqb, BH, qb, bh);
         const int b = bh / H, h = bh % H, row0 = b * T;
@@ -849,7 +915,7 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc = att_idesc(HD, 1) | (1u << 15);  // N = 64, A and B MN-major
       uint32_t g = 0, t = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < nitems; w += gridDim.x, ++t) {
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k), ++t) {
         int qb, bh;
         item_desc(w, nqb, BH, qb, bh);
         const uint32_t ab = t & 1u;
@@ -885,7 +951,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t t = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < nitems; w += gridDim.x, ++t) {
+    for (int k = 0, w = snake_item(0); w < nitems; w = snake_item(++k), ++t) {
       int qb, bh;
       item_desc(w, nqb, BH, qb, bh);
       const int b = bh / H, h = bh % H, row0 = b * T;
@@ -978,15 +1044,20 @@ static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16*
   const int items = ((T + BT - 1) / BT) * B * H;
   const int grid = items < num_sms_attn() ? items : num_sms_attn();
   if (ds != nullptr) {
+    // (the TMA row coordinates of the dS tiles are 32-bit)
+    if (backward_ds_elems(B, T, H) / BT >= (1L << 31)) return cudaErrorInvalidValue;
     CUtensorMap tds;
     if (make_tmap(&tds, ds, BT, backward_ds_elems(B, T, H) / BT, BT, 64, 64) != 0) return cudaErrorInvalidValue;
     const long n = (long)B * ((T + BT - 1) / BT) * BT * H;
-    ld_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
-    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, ds, T, H, B * H, scale, sl2);
+    if (((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(dout)) & 31) == 0)
+      ld_kernel<true><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
+    else
+      ld_kernel<false><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
+    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, tds, ld, dqkv, colsum, 1, T, H, B * H, scale, sl2);
     dq_mma_kernel<<<grid, 192, DQM_SMEM, st>>>(tds, tq, dqkv, colsum, T, H, B * H, scale);
   } else {
     dq_kernel<<<grid, BW_THREADS, DQ_SMEM, st>>>(tq, td, out, lse, ld, dqkv, colsum, T, H, B * H, scale, sl2);
-    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, ld, dqkv, colsum, nullptr, T, H, B * H, scale, sl2);
+    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, tq, ld, dqkv, colsum, 0, T, H, B * H, scale, sl2);
   }
   return cudaGetLastError();
 }

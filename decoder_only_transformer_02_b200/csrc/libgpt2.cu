@@ -260,6 +260,29 @@ int gpt2_get_embed_keys(gpt2_t* h, uint32_t* dst) {
 
 int64_t gpt2_kernel_launches(const gpt2_t* h) { return h ? h->launches : -1; }
 
+int gpt2_check_guards(gpt2_t* h, int64_t* n_bad) {
+  if (h == nullptr || n_bad == nullptr) return GPT2_EINVAL;
+  if (cudaStreamSynchronize(h->stream) != cudaSuccess) return set_err(h, GPT2_ECUDA, "stream synchronise");
+  if (h->side_stream && cudaStreamSynchronize(h->side_stream) != cudaSuccess)
+    return set_err(h, GPT2_ECUDA, "stream synchronise");
+  int64_t bad = 0;
+  unsigned char buf[GUARD_BYTES];
+  for (const auto& g : h->guards) {
+    if (cudaMemcpy(buf, static_cast<const uint8_t*>(g.first) + g.second, GUARD_BYTES, cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      return set_err(h, GPT2_ECUDA, "guard read");
+    for (size_t i = 0; i < GUARD_BYTES; ++i) bad += buf[i] != GUARD_BYTE;
+  }
+  *n_bad = bad;
+  return GPT2_OK;
+}
+
+int gpt2_debug_overwrite_guard(gpt2_t* h, int index) {
+  if (h == nullptr || index < 0 || index >= (int)h->guards.size()) return GPT2_EINVAL;
+  const auto& g = h->guards[index];
+  return cudaMemset(static_cast<uint8_t*>(g.first) + g.second, 0, 1) == cudaSuccess ? GPT2_OK : GPT2_ECUDA;
+}
+
 int gpt2_set_graphs(gpt2_t* h, int enable) {
   if (h == nullptr) return GPT2_EINVAL;
   h->use_graphs = enable != 0;

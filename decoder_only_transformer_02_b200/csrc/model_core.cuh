@@ -32,6 +32,8 @@ struct gpt2 {
   size_t es = 4;  // bytes per activation element (2 in bf16 mode)
   cudaStream_t stream = nullptr;
   std::string err = "ok";
+  // guard bytes after every device allocation: (allocation, offset of its guard)
+  std::vector<std::pair<void*, size_t>> guards;
   int64_t launches = 0;
 
   // parameters, flat
@@ -193,13 +195,21 @@ static void build_tensor_table(gpt2* h) {
   h->nparams = off;
 }
 
+// Every device allocation is rounded up to 256 bytes and followed by
+// GUARD_BYTES of GUARD_BYTE: a kernel that writes past the end of a buffer
+// changes them, and gpt2_check_guards reports it.
+constexpr size_t GUARD_BYTES = 256;
+constexpr unsigned char GUARD_BYTE = 0xA5;
 static int dev_alloc(gpt2* h, void** p, size_t bytes) {
-  if (bytes == 0) bytes = 16;
-  cudaError_t e = cudaMalloc(p, bytes);
+  const size_t body = ((bytes == 0 ? 16 : bytes) + 255) & ~size_t(255);
+  cudaError_t e = cudaMalloc(p, body + GUARD_BYTES);
+  if (e == cudaSuccess) e = cudaMemset(static_cast<uint8_t*>(*p) + body, GUARD_BYTE, GUARD_BYTES);
   if (e != cudaSuccess) {
+    if (*p) cudaFree(*p);
     *p = nullptr;
     return set_err(h, GPT2_ENOMEM, std::string("cudaMalloc(") + std::to_string(bytes) + "): " + cudaGetErrorString(e));
   }
+  h->guards.emplace_back(*p, body);
   return GPT2_OK;
 }
 #define ALLOC(h, ptr, bytes)                                                    \

@@ -28,7 +28,8 @@ EXPORTED = [
     "gpt2_last_error", "gpt2_attention_forward", "gpt2_attention_backward", "gpt2_attention_workspace_floats",
     "gpt2_matmul_bf16", "gpt2_matmul_workspace_bytes", "gpt2_set_timing", "gpt2_get_timing",
     "gpt2_attention_backward_noalloc", "gpt2_set_graphs", "gpt2_check_device_error", "gpt2_set_wait_limit_ns",
-    "gpt2_prefill", "gpt2_decode_step", "gpt2_get_decode_logits",
+    "gpt2_prefill", "gpt2_decode_step", "gpt2_get_decode_logits", "gpt2_check_guards",
+    "gpt2_debug_overwrite_guard",
 ]
 ATTN_NOALLOC_MAX_ROWS = 1 << 19  # padded (batch, head, position) rows
 KCLASSES = ["matmul", "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd", "cross_entropy",
@@ -83,6 +84,8 @@ def load_library():
         "gpt2_last_loss": (I, [P, P]),
         "gpt2_get_embed_keys": (I, [P, P]),
         "gpt2_kernel_launches": (L, [P]),
+        "gpt2_check_guards": (I, [P, P]),
+        "gpt2_debug_overwrite_guard": (I, [P, I]),
         "gpt2_last_error": (ctypes.c_char_p, [P]),
         "gpt2_attention_forward": (I, [P, P, P, I, I, I, P]),
         "gpt2_attention_backward": (I, [P, P, P, P, P, P, I, I, I, P]),
@@ -263,6 +266,16 @@ class GPT2:
     @property
     def kernel_launches(self) -> int:
         return int(self._lib.gpt2_kernel_launches(self._h))
+
+    def check_guards(self) -> int:
+        """Number of guard bytes after the handle's device buffers that some
+        kernel overwrote (0 when every write stayed inside its buffer)."""
+        n = ctypes.c_int64(0)
+        self._check(self._lib.gpt2_check_guards(self._h, ctypes.byref(n)))
+        return int(n.value)
+
+    def debug_overwrite_guard(self, index: int):
+        self._check(self._lib.gpt2_debug_overwrite_guard(self._h, index))
 
     def get_params(self) -> np.ndarray:
         a = np.empty(self.num_params, dtype=np.float32)

@@ -171,6 +171,16 @@ int gpt2_last_loss(gpt2_t* h, float* h_loss);   /* mean loss of the last forward
 int gpt2_get_embed_keys(gpt2_t* h, uint32_t* h_dst);
 /* Number of kernels this handle has launched since creation. */
 int64_t gpt2_kernel_launches(const gpt2_t* h);
+/* Guard bytes (no counterpart in the paper: a check of this library's own
+ * kernels).  Every device buffer the handle allocates is rounded up to 256
+ * bytes and followed by 256 guard bytes of 0xA5.  Waits for the handle's
+ * work, then *n_bad = the number of guard bytes that no longer hold 0xA5
+ * (0 unless some kernel wrote past the end of a buffer). */
+int gpt2_check_guards(gpt2_t* h, int64_t* n_bad);
+/* Test hook for the check above: overwrites one byte of the guard of the
+ * index-th allocation (in allocation order).  GPT2_EINVAL for an index out of
+ * range. */
+int gpt2_debug_overwrite_guard(gpt2_t* h, int index);
 
 /* ---- measurement support ----
  * With timing enabled, every operation this handle enqueues is bracketed by a

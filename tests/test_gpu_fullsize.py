@@ -72,3 +72,5 @@ def test_fullsize_gradients_repeated_sequence(setup):
     assert not bad, bad
     norm = m.adamw_step(6e-4, want_norm=True)
     assert abs(norm - O.grad_norm(gref)) / O.grad_norm(gref) < 1e-2
+    # every kernel of the step stayed inside its buffers
+    assert m.check_guards() == 0

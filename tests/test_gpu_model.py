@@ -357,3 +357,38 @@ def test_nonfinite_gradient_skips_update():
     np.testing.assert_array_equal(np.isnan(after), np.isnan(before))
     np.testing.assert_array_equal(after[~np.isnan(after)], before[~np.isnan(before)])
     assert m.get_adam_state()[2] == 0
+
+
+# ---------------------------------------------------------- guard bytes
+
+def test_guard_bytes_intact_after_steps_and_generation():
+    """Every device buffer is followed by guard bytes: after bf16 and fp32
+    optimizer steps at ragged shapes and a generation run, none has changed."""
+    G, O, cfg, m = make(BF_CFG, 3, 200, 1)
+    (tok, tgt), = batch("uniform", 500, 3, 200, 7)
+    for k in range(2):
+        m.forward_backward(dev(tok), dev(tgt), 0.5)
+    m.adamw_step(6e-4)
+    nxt = torch.empty(3, dtype=torch.int32, device="cuda")
+    m.prefill(dev(tok[:, :37]), nxt, temperature=0.8, top_k=5, seed=11)
+    for pos in range(37, 45):
+        m.decode_step(nxt.clone(), pos, nxt, temperature=0.8, top_k=5, seed=11)
+    assert m.check_guards() == 0
+    m.close()
+    G, O, cfg, m = make(TINY_CFG, 4, 64, 0)
+    (tok, tgt), = batch("uniform", 512, 4, 64, 8)
+    m.forward_backward(dev(tok), dev(tgt), 1.0)
+    m.adamw_step(6e-4)
+    assert m.check_guards() == 0
+    m.close()
+
+
+def test_guard_check_reports_an_overwritten_guard():
+    G, O, cfg, m = make(TINY_CFG, 4, 64, 0)
+    assert m.check_guards() == 0
+    m.debug_overwrite_guard(3)
+    assert m.check_guards() == 1
+    with pytest.raises(G.GPT2Error):
+        m.debug_overwrite_guard(1 << 20)
+    m.close()
+
