@@ -200,133 +200,163 @@ __global__ void ln_fwd_kernel(const float* __restrict__ x, const float* __restri
   }
 }
 
-// LayerNorm backward fused with the residual stream.  One warp per row:
+// LayerNorm backward fused with the residual stream, per row:
 //   dxhat = dy*g ; dx = rstd*(dxhat - mean(dxhat) - xhat*mean(dxhat*xhat))
 //   dres = (accumulate ? dres : 0) + dx     (fp32, in place)   and a bf16 copy
 // and per-block partial column sums (fixed row ranges, fixed order) of
 //   dy*xhat (-> dgamma), dy (-> dbeta), dres_out (-> the bias gradient of the
 //   linear layer whose output is this residual point).
-// The column accumulators live in shared memory, one private slice per warp
-// (each lane owns its columns: no conflicts, no atomics), which keeps the
-// register count low enough for two CTAs per SM.  Dynamic shared memory:
-// 3 * C * LN_BWD_WARPS floats.
-constexpr int LN_BWD_WARPS = 4;
-template <int NV, typename TI>
-__device__ __forceinline__ void ln_bwd_load(const TI* __restrict__ dy, const float* __restrict__ x,
-                                            const float* __restrict__ dres, long row, int lane, int accumulate,
-                                            float4 (&xv)[NV], float4 (&dyv)[NV], float4 (&rv)[NV]) {
-  constexpr int C = 128 * NV;
-  const float4* xr = reinterpret_cast<const float4*>(x + row * C) + lane;
-  const float4* dr = reinterpret_cast<const float4*>(dres + row * C) + lane;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    xv[i] = xr[32 * i];
-    if constexpr (sizeof(TI) == 2) {
-      const uint2 u = reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(dy) + row * C)[lane + 32 * i];
-      const float2 a0 = unpack_bf16x2(u.x), a1 = unpack_bf16x2(u.y);
-      dyv[i] = make_float4(a0.x, a0.y, a1.x, a1.y);
-    } else {
-      dyv[i] = (reinterpret_cast<const float4*>(reinterpret_cast<const float*>(dy) + row * C) + lane)[32 * i];
-    }
-    rv[i] = accumulate ? dr[32 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
-// Software-pipelined: the loads of a warp's next row are issued before the
-// reductions of its current row, so two rows per warp are in flight.
-template <int NV, typename TI>
-__global__ void __launch_bounds__(LN_BWD_WARPS * 32, 2) ln_bwd_kernel(const TI* __restrict__ dy, const float* __restrict__ x,
-                                                     const float* __restrict__ mean, const float* __restrict__ rstd,
-                                                     const float* __restrict__ gam, float* __restrict__ dres,
-                                                     bf16* __restrict__ dres_bf, int M, int rows_per_block,
-                                                     int accumulate, float* __restrict__ part) {
-  constexpr int C = 128 * NV;
-  constexpr int C4 = C / 4;
-  extern __shared__ float4 ln_acc[];  // [warp][3][C4]
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float4* acc = ln_acc + warp * 3 * C4;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c4 = lane + 32 * i;
-    acc[c4] = acc[C4 + c4] = acc[2 * C4 + c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+// A CTA owns a fixed range of rows.  One producer thread streams them into
+// shared memory with bulk asynchronous copies (dy, x and the incoming dres of
+// LN_BWD_WARPS rows per stage, LnBwd<NV>::STAGES stages), so the bytes in
+// flight do not depend on registers; each compute warp takes one row of a
+// stage, reads it from shared memory, writes dres / dres_bf to global memory,
+// and keeps its columns' sums in registers.  At the end the warps' sums are
+// combined in warp order.  Rows per CTA: a multiple of LN_BWD_WARPS.
+constexpr int LN_BWD_WARPS = 7;  // compute warps (with the producer: 256 threads, so 255 registers each)
+template <int NV>
+struct LnBwd {
+  static constexpr int C = 128 * NV;
+  static constexpr int ROW = 3 * C;                     // floats per staged row: dy, x, dres
+  static constexpr int STAGES = NV <= 6 ? 3 : 2;
+  static constexpr int STAGE_FLOATS = LN_BWD_WARPS * ROW;
+  static size_t smem_bytes(int rpb) { return (size_t)STAGES * STAGE_FLOATS * 4 + (size_t)2 * rpb * 4 + 2 * STAGES * 8; }
+};
+template <int NV>
+__global__ void __launch_bounds__(32 * (LN_BWD_WARPS + 1), 1)
+    ln_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
+                  const float* __restrict__ rstd, const float* __restrict__ gam, float* __restrict__ dres,
+                  bf16* __restrict__ dres_bf, int M, int rows_per_block, int accumulate, float* __restrict__ part) {
+  using L = LnBwd<NV>;
+  constexpr int C = L::C, S = L::STAGES, W = LN_BWD_WARPS;
+  extern __shared__ float4 ln_smem4[];
+  float* stage = reinterpret_cast<float*>(ln_smem4);  // [S][W][dy | x | dres]
+  float* mr = stage + S * L::STAGE_FLOATS;              // mean [rows_per_block], rstd [rows_per_block]
+  uint64_t* full = reinterpret_cast<uint64_t*>(mr + 2 * rows_per_block);
+  uint64_t* empty = full + S;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long r0 = (long)blockIdx.x * rows_per_block;
-  const long r1 = min((long)M, r0 + rows_per_block);
-  float4 xv[NV], dyv[NV], rv[NV];
-  long row = r0 + warp;
-  float mu = 0.f, rs = 0.f;
-  if (row < r1) {
-    ln_bwd_load<NV, TI>(dy, x, dres, row, lane, accumulate, xv, dyv, rv);
-    mu = mean[row];
-    rs = rstd[row];
+  const int nrows = (int)(min((long)M, r0 + rows_per_block) - r0);
+  const int nbatch = (nrows + W - 1) / W;
+  for (int i = threadIdx.x; i < nrows; i += blockDim.x) {
+    mr[i] = mean[r0 + i];
+    mr[rows_per_block + i] = rstd[r0 + i];
   }
-  for (; row < r1; row += LN_BWD_WARPS) {
-    // next row's loads first
-    const long nrow = row + LN_BWD_WARPS;
-    float4 xn[NV], dyn[NV], rn[NV];
-    float mun = 0.f, rsn = 0.f;
-    if (nrow < r1) {
-      ln_bwd_load<NV, TI>(dy, x, dres, nrow, lane, accumulate, xn, dyn, rn);
-      mun = mean[nrow];
-      rsn = rstd[nrow];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tcg::mbar_init(&full[s], 1);
+      tcg::mbar_init(&empty[s], W);
     }
-    float4* dr = reinterpret_cast<float4*>(dres + row * C) + lane;
-    float s1 = 0.f, s2 = 0.f;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  float4 adg[NV], adb[NV], adr[NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const float4 g = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
-      xv[i] = make_float4((xv[i].x - mu) * rs, (xv[i].y - mu) * rs, (xv[i].z - mu) * rs, (xv[i].w - mu) * rs);
-      const float d0 = dyv[i].x * g.x, d1 = dyv[i].y * g.y, d2 = dyv[i].z * g.z, d3 = dyv[i].w * g.w;
-      s1 += d0 + d1 + d2 + d3;
-      s2 += d0 * xv[i].x + d1 * xv[i].y + d2 * xv[i].z + d3 * xv[i].w;
+  for (int i = 0; i < NV; ++i) adg[i] = adb[i] = adr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == W) {
+    if (lane == 0) {
+      // ------------------------------------------------------ producer
+      bool ok = true;
+      int issued = 0;
+      for (int k = 0; k < nbatch; ++k, ++issued) {
+        const int s = k % S;
+        if (!tcg::mbar_wait(&empty[s], ((k / S) & 1u) ^ 1u)) {
+          ok = false;
+          break;
+        }
+        const int nr = min(W, nrows - k * W);
+        tcg::mbar_expect_tx(&full[s], (uint32_t)(nr * (accumulate ? 3 : 2) * C * 4));
+        for (int w = 0; w < nr; ++w) {
+          const long row = r0 + (long)k * W + w;
+          float* dst = stage + (long)s * L::STAGE_FLOATS + w * L::ROW;
+          tcfa::bulk_load(tcg::smem_u32(dst), dy + row * C, C * 4, &full[s]);
+          tcfa::bulk_load(tcg::smem_u32(dst + C), x + row * C, C * 4, &full[s]);
+          if (accumulate) tcfa::bulk_load(tcg::smem_u32(dst + 2 * C), dres + row * C, C * 4, &full[s]);
+        }
+      }
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      tcfa::drain_ring(full, S, (uint32_t)issued);
     }
-    s1 = warp_sum(s1) * (1.f / C);
-    s2 = warp_sum(s2) * (1.f / C);
+  } else {
+    // ------------------------------------------------- compute warps
+    float4 g[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) g[i] = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
+    bool ok = true;
+    for (int k = 0; k < nbatch; ++k) {
+      const int s = k % S;
+      if (!tcfa::warp_wait(&full[s], (k / S) & 1u)) {
+        ok = false;
+        break;
+      }
+      const int ri = k * W + warp;
+      if (ri < nrows) {
+        const long row = r0 + ri;
+        const float4* src = reinterpret_cast<const float4*>(stage + (long)s * L::STAGE_FLOATS + warp * L::ROW);
+        const float mu = mr[ri], rs = mr[rows_per_block + ri];
+        float4 dyv[NV], xv[NV];
+        float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          dyv[i] = src[lane + 32 * i];
+          const float4 xr = src[C / 4 + lane + 32 * i];
+          xv[i] = make_float4((xr.x - mu) * rs, (xr.y - mu) * rs, (xr.z - mu) * rs, (xr.w - mu) * rs);
+          const float d0 = dyv[i].x * g[i].x, d1 = dyv[i].y * g[i].y, d2 = dyv[i].z * g[i].z, d3 = dyv[i].w * g[i].w;
+          s1 += d0 + d1 + d2 + d3;
+          s2 += d0 * xv[i].x + d1 * xv[i].y + d2 * xv[i].z + d3 * xv[i].w;
+        }
+        s1 = warp_sum(s1) * (1.f / C);
+        s2 = warp_sum(s2) * (1.f / C);
+        float4* dr = reinterpret_cast<float4*>(dres + row * C) + lane;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const int c4 = lane + 32 * i;
+          const float4 rv = accumulate ? src[C / 2 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 o;
+          o.x = rv.x + rs * (dyv[i].x * g[i].x - s1 - xv[i].x * s2);
+          o.y = rv.y + rs * (dyv[i].y * g[i].y - s1 - xv[i].y * s2);
+          o.z = rv.z + rs * (dyv[i].z * g[i].z - s1 - xv[i].z * s2);
+          o.w = rv.w + rs * (dyv[i].w * g[i].w - s1 - xv[i].w * s2);
+          dr[32 * i] = o;
+          if (dres_bf != nullptr)
+            reinterpret_cast<uint2*>(dres_bf + row * C)[c4] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+          adg[i].x += dyv[i].x * xv[i].x;
+          adg[i].y += dyv[i].y * xv[i].y;
+          adg[i].z += dyv[i].z * xv[i].z;
+          adg[i].w += dyv[i].w * xv[i].w;
+          adb[i].x += dyv[i].x;
+          adb[i].y += dyv[i].y;
+          adb[i].z += dyv[i].z;
+          adb[i].w += dyv[i].w;
+          adr[i].x += o.x;
+          adr[i].y += o.y;
+          adr[i].z += o.z;
+          adr[i].w += o.w;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tcg::mbar_arrive(&empty[s]);
+    }
+    if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+  }
+  __syncthreads();  // every row is done and every copy has landed: the stages are free
+  // combine the warps' column sums in warp order
+  float4* acc = reinterpret_cast<float4*>(stage);  // [W][3][C/4]
+  if (warp < W) {
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c4 = lane + 32 * i;
-      const float4 g = reinterpret_cast<const float4*>(gam)[c4];
-      float4 o;
-      o.x = rv[i].x + rs * (dyv[i].x * g.x - s1 - xv[i].x * s2);
-      o.y = rv[i].y + rs * (dyv[i].y * g.y - s1 - xv[i].y * s2);
-      o.z = rv[i].z + rs * (dyv[i].z * g.z - s1 - xv[i].z * s2);
-      o.w = rv[i].w + rs * (dyv[i].w * g.w - s1 - xv[i].w * s2);
-      dr[32 * i] = o;
-      if (dres_bf != nullptr)
-        reinterpret_cast<uint2*>(dres_bf + row * C)[c4] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
-      float4 a = acc[c4], b = acc[C4 + c4], d = acc[2 * C4 + c4];
-      a.x += dyv[i].x * xv[i].x;
-      a.y += dyv[i].y * xv[i].y;
-      a.z += dyv[i].z * xv[i].z;
-      a.w += dyv[i].w * xv[i].w;
-      b.x += dyv[i].x;
-      b.y += dyv[i].y;
-      b.z += dyv[i].z;
-      b.w += dyv[i].w;
-      d.x += o.x;
-      d.y += o.y;
-      d.z += o.z;
-      d.w += o.w;
-      acc[c4] = a;
-      acc[C4 + c4] = b;
-      acc[2 * C4 + c4] = d;
+      acc[(warp * 3 + 0) * (C / 4) + c4] = adg[i];
+      acc[(warp * 3 + 1) * (C / 4) + c4] = adb[i];
+      acc[(warp * 3 + 2) * (C / 4) + c4] = adr[i];
     }
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      xv[i] = xn[i];
-      dyv[i] = dyn[i];
-      rv[i] = rn[i];
-    }
-    mu = mun;
-    rs = rsn;
   }
   __syncthreads();
-  // combine the warps' slices in warp order
-  const float* af = reinterpret_cast<const float*>(ln_acc);
+  const float* af = reinterpret_cast<const float*>(acc);
   for (int idx = threadIdx.x; idx < 3 * C; idx += blockDim.x) {
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < LN_BWD_WARPS; ++w) t += af[w * 3 * C + idx];
+    for (int w = 0; w < W; ++w) t += af[w * 3 * C + idx];
     part[(long)blockIdx.x * 3 * C + idx] = t;
   }
 }

@@ -231,11 +231,12 @@ static void free_all(gpt2* h) {
     if (p) cudaFree(p);
 }
 
-// rows handled per CTA by the LayerNorm backward: one wave of 2 CTAs per SM
+// rows handled per CTA by the LayerNorm backward: one CTA per SM, a whole
+// number of stages of k::LN_BWD_WARPS rows
 static int ln_rows_per_block(long M) {
-  long r = (M + 295) / 296;
-  r = (r + 3) / 4 * 4;
-  return (int)(r < 4 ? 4 : r);
+  long r = (M + 147) / 148;
+  r = (r + k::LN_BWD_WARPS - 1) / k::LN_BWD_WARPS * k::LN_BWD_WARPS;
+  return (int)r;
 }
 // rows per CTA of the column-sum kernel: at most 64 row blocks
 static int colsum_rows_per_block(long M) {

@@ -30,6 +30,18 @@ static int op_ln_fwd(gpt2* h, const float* x, size_t goff, size_t boff, void* y,
   return ln_fwd_dispatch<float>(h, x, h->P32(goff), h->P32(boff), (float*)y, mean, rstd, M);
 }
 
+// the LayerNorm backward's dynamic shared memory limit (set once per device
+// to the most a CTA may have)
+constexpr size_t LN_BWD_SMEM_MAX = 227 * 1024;
+template <int NV>
+static bool ln_bwd_attr() {
+  static DeviceOnce once;
+  return run_once_per_device(once, [] {
+           return cudaFuncSetAttribute(k::ln_bwd_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)LN_BWD_SMEM_MAX);
+         }) == cudaSuccess;
+}
+
 // LayerNorm backward into the running residual gradient h->dres.  dy is fp32
 // [M, C].  Adds dgamma, dbeta and (when dbias_off != NO_OFF) the column sums of
 // the resulting residual gradient into the grads.
@@ -39,11 +51,12 @@ static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean
   const int rpb = ln_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
   bf16* dbf = h->prec == GPT2_BF16 ? h->dres_bf : nullptr;
-  const size_t smem = (size_t)3 * h->C * k::LN_BWD_WARPS * sizeof(float);
   switch (h->C / 128) {
 #define LNB(NV)                                                                                                     \
   case NV:                                                                                                          \
-    k::ln_bwd_kernel<NV, float><<<nblk, k::LN_BWD_WARPS * 32, smem, h->stream>>>(                                 \
+    if (k::LnBwd<NV>::smem_bytes(rpb) > LN_BWD_SMEM_MAX) return set_err(h, GPT2_EINVAL, "layernorm: rows");     \
+    if (!ln_bwd_attr<NV>()) return set_err(h, GPT2_ECUDA, "layernorm backward shared memory");                  \
+    k::ln_bwd_kernel<NV><<<nblk, (k::LN_BWD_WARPS + 1) * 32, k::LnBwd<NV>::smem_bytes(rpb), h->stream>>>(       \
         dy, x, mean, rstd, h->P32(goff), h->dres, dbf, (int)M, rpb, accumulate, h->ln_part);                        \
     break;
     LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
