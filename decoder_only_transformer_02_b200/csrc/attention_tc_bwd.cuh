@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       if (q < T) store_row16(dqkv + ((long)row0 + q) * (3L * C) + h * HD + cq * 16, a, scale);
       if (colsum) {
         const float tot = warp_colsum16(cs, lane);
-        if (lane < 16) colsum[(((long)b * nqb + qb) * 4 + qw) * (3L * C) + h * HD + cq * 16 + lane] = tot;
+        if (lane < 16) colsum[(((long)b * nqb + qb) * 4 + qw) * (3L * C) + h * HD + cq * 16 + lane] += tot;
       }
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
@@ -747,8 +747,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         for (int i = 0; i < 16; ++i) cs[i] = key < T ? __uint_as_float(av[i]) : 0.f;
         const float tv = warp_colsum16(cs, lane);
         if (lane < 16) {
-          colsum[prow + C + h * HD + cq * 16 + lane] = tk;
-          colsum[prow + 2 * C + h * HD + cq * 16 + lane] = tv;
+          colsum[prow + C + h * HD + cq * 16 + lane] += tk;
+          colsum[prow + 2 * C + h * HD + cq * 16 + lane] += tv;
         }
       }
     }
@@ -766,7 +766,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
 // The per-query values the backward kernels stream: lse*log2(e) and
 // D = sum_d dO[q,d] O[q,d], padded to whole 128-query blocks (+inf and 0 past
 // T), in ld[((b*H + h)*nqb + qb)*LD_FLOATS + r] and [... + BT + r].  One thread
-// per (padded row, head), heads fastest so that a warp reads contiguous rows.
+// per (batch, head, padded position), positions fastest: a thread reads its
+// row's 128 bytes in whole sectors and a warp writes 32 consecutive floats.
 // The sum runs in the same order as in dq_kernel (four chains over pairs of
 // columns), so either route gives the same bits.  V32: out and dout are
 // 32-byte aligned (rows are read as 32-byte vectors), else 16-byte vectors.
@@ -778,9 +779,9 @@ __global__ void __launch_bounds__(256) ld_kernel(const bf16* __restrict__ out, c
   const long n = (long)B * nqb * BT * H;
   const long gi = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gi >= n) return;
-  const int h = (int)(gi % H);
-  const long m = gi / H;
-  const int b = (int)(m / ((long)nqb * BT)), q = (int)(m % ((long)nqb * BT));
+  const int q = (int)(gi % ((long)nqb * BT));
+  const long bhi = gi / ((long)nqb * BT);
+  const int h = (int)(bhi % H), b = (int)(bhi / H);
   const int C = H * HD;
   float l2 = INFINITY, dq_ = 0.f;
   if (q < T) {
@@ -983,8 +984,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) cs[i] = q < T ? __uint_as_float(a1[i]) * scale : 0.f;
         const float t1 = warp_colsum32(cs, lane);
-        colsum[prow + lane] = t0;
-        colsum[prow + 32 + lane] = t1;
+        colsum[prow + lane] += t0;
+        colsum[prow + 32 + lane] += t1;
       }
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
@@ -1012,8 +1013,8 @@ static inline long backward_colsum_rows(int B, int T) { return (long)B * ((T + B
 
 // The attention backward.  ld: fp32 scratch of backward_scratch_floats(B, T,
 // H) elements, 16-byte aligned.  colsum (may be null): [backward_colsum_rows(B,
-// T)][3C] fp32 partial column sums of dqkv (summing them over the rows gives
-// the qkv bias gradient).
+// T)][3C] fp32 partial column sums of dqkv, added to what it holds (summing
+// them over the rows gives the qkv bias gradient).
 //  ds given (backward_ds_elems(B, T, H) bf16, 16-byte aligned): ld_kernel forms
 //     lse*log2(e) and D, dkdv_kernel forms P and dS once per score and stores
 //     dS, dq_mma_kernel reads it back for dQ (three launches).

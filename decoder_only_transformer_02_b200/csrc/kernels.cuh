@@ -86,32 +86,49 @@ __global__ void sort_keys_kernel(const int32_t* __restrict__ tok, int M, int V, 
 }
 
 // Stage 1 of the deterministic scatter-add.  Sorted entries are cut into
-// chunks of CH; chunk c sums each run of equal tokens it holds (positions in
-// ascending order) and writes the run's sum to part[first sorted index of the
-// run].  dx0 is fp32 [M, C]; one CTA per chunk, threads over columns.
+// chunks of EMB_CH; chunk c sums each run of equal tokens it holds (positions
+// in ascending order) and writes the run's sum to part[first sorted index of
+// the run].  dx0 is fp32 [M, C]; one CTA per chunk, one thread per 4 columns
+// (blockDim >= C/4); the chunk's keys sit in shared memory and eight rows'
+// loads are in flight at a time.
 constexpr int EMB_CH = 32;
 __global__ void embed_bwd_partial_kernel(const uint32_t* __restrict__ keys, const float* __restrict__ dx, int M, int C,
                                          float* __restrict__ part) {
+  __shared__ uint32_t ks[EMB_CH];
   const int c0 = blockIdx.x * EMB_CH;
-  const int c1 = min(M, c0 + EMB_CH);
-  for (int col = threadIdx.x; col < C; col += blockDim.x) {
-    int run_start = c0;
-    float acc = 0.f;
-    for (int s = c0; s < c1; ++s) {
-      const uint32_t key = keys[s];
-      acc += dx[(long)(key & 0xffffu) * C + col];
-      const bool last = (s + 1 == c1) || ((keys[s + 1] >> 16) != (key >> 16));
-      if (last) {
-        part[(long)run_start * C + col] = acc;
-        acc = 0.f;
-        run_start = s + 1;
+  const int n = min(EMB_CH, M - c0);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) ks[i] = keys[c0 + i];
+  __syncthreads();
+  const int c4 = threadIdx.x;
+  if (c4 >= C / 4) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int run_start = 0;
+  for (int s0 = 0; s0 < n; s0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (s0 + j < n) v[j] = reinterpret_cast<const float4*>(dx + (long)(ks[s0 + j] & 0xffffu) * C)[c4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int s = s0 + j;
+      if (s < n) {
+        acc.x += v[j].x;
+        acc.y += v[j].y;
+        acc.z += v[j].z;
+        acc.w += v[j].w;
+        if (s + 1 == n || (ks[s + 1] >> 16) != (ks[s] >> 16)) {
+          reinterpret_cast<float4*>(part + (long)(c0 + run_start) * C)[c4] = acc;
+          acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          run_start = s + 1;
+        }
       }
     }
   }
 }
 
-// Stage 2: one CTA per sorted index that starts a token's segment; sums the
-// run partials of that segment (in sorted order) into dwte[token].
+// Stage 2: one CTA per sorted index (launched with a grid of M); the CTAs at a
+// token's first sorted index sum the run partials of that token's segment (in
+// sorted order) into dwte[token].  One thread per 4 columns.
 __global__ void embed_bwd_reduce_kernel(const uint32_t* __restrict__ keys, const float* __restrict__ part, int M, int C,
                                         int V, float* __restrict__ dwte) {
   for (int s = blockIdx.x; s < M; s += gridDim.x) {
@@ -129,24 +146,62 @@ __global__ void embed_bwd_reduce_kernel(const uint32_t* __restrict__ keys, const
         hi = mid;
     }
     const int e = lo;
-    for (int col = threadIdx.x; col < C; col += blockDim.x) {
-      float acc = 0.f;
+    for (int c4 = threadIdx.x; c4 < C / 4; c4 += blockDim.x) {
       // run partials start at s and at each chunk boundary inside [s, e)
-      acc += part[(long)s * C + col];
+      float4 acc = reinterpret_cast<const float4*>(part + (long)s * C)[c4];
 #pragma unroll 4
-      for (int cb = (s / EMB_CH + 1) * EMB_CH; cb < e; cb += EMB_CH) acc += part[(long)cb * C + col];
-      dwte[(long)tokn * C + col] += acc;
+      for (int cb = (s / EMB_CH + 1) * EMB_CH; cb < e; cb += EMB_CH) {
+        const float4 v = reinterpret_cast<const float4*>(part + (long)cb * C)[c4];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      float4* d = reinterpret_cast<float4*>(dwte + (long)tokn * C) + c4;
+      const float4 o = *d;
+      *d = make_float4(o.x + acc.x, o.y + acc.y, o.z + acc.z, o.w + acc.w);
     }
   }
 }
 
-// dwpe[t] += sum_b dx0[b,t]
+
+// g[i] += slots[0][i] + slots[1][i] + ... (in split order), and the slots
+// are cleared for the next accumulation.  n % 4 == 0.
+__global__ void slot_fold_kernel(float* __restrict__ g, float* __restrict__ slots, long n, int splits) {
+  const long n4 = n / 4;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(g)[i];
+    for (int s = 0; s < splits; ++s) {
+      float4* q = reinterpret_cast<float4*>(slots + s * n) + i;
+      const float4 v = *q;
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+      *q = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    reinterpret_cast<float4*>(g)[i] = acc;
+  }
+}
+
+// dwpe[t] += sum_b dx0[b,t] (in batch order); one thread per 4 columns of a
+// position
 __global__ void wpe_bwd_kernel(const float* __restrict__ dx, int B, int T, int C, float* __restrict__ dwpe) {
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < (long)T * C; i += (long)gridDim.x * blockDim.x) {
-    const long t = i / C, c = i % C;
-    float acc = 0.f;
-    for (int b = 0; b < B; ++b) acc += dx[((long)b * T + t) * C + c];
-    dwpe[t * C + c] += acc;
+  const int C4 = C / 4;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < (long)T * C4; i += (long)gridDim.x * blockDim.x) {
+    const long t = i / C4, c = i % C4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int b = 0; b < B; ++b) {
+      const float4 v = reinterpret_cast<const float4*>(dx + ((long)b * T + t) * C)[c];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    float4* d = reinterpret_cast<float4*>(dwpe + t * C) + c;
+    const float4 o = *d;
+    *d = make_float4(o.x + acc.x, o.y + acc.y, o.z + acc.z, o.w + acc.w);
   }
 }
 
@@ -357,7 +412,7 @@ __global__ void __launch_bounds__(32 * (LN_BWD_WARPS + 1), 1)
     float t = 0.f;
 #pragma unroll
     for (int w = 0; w < W; ++w) t += af[w * 3 * C + idx];
-    part[(long)blockIdx.x * 3 * C + idx] = t;
+    part[(long)blockIdx.x * 3 * C + idx] += t;  // (accumulates over the micro-steps)
   }
 }
 
@@ -445,7 +500,7 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 #pragma unroll
     for (int w = 0; w < 8; ++w) t += red[w][i];
     const int col = blockIdx.x * 32 * VEC + i;
-    if (col < N) part[(long)blockIdx.y * N + col] = t;
+    if (col < N) part[(long)blockIdx.y * N + col] += t;  // (accumulates over the micro-steps)
   }
 }
 

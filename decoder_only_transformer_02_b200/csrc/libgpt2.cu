@@ -109,6 +109,7 @@ int gpt2_forward_backward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int
 
 int gpt2_zero_grad(gpt2_t* h) {
   if (h == nullptr) return GPT2_EINVAL;
+  RET_IF(clear_accumulators(h));
   CU_CHECK(h, cudaMemsetAsync(h->grads, 0, h->nparams * 4, h->stream));
   return GPT2_OK;
 }
@@ -132,6 +133,7 @@ int gpt2_train_step(gpt2_t* h, const int32_t* h_tok, const int32_t* h_tgt, int n
   if (h_tok == nullptr || h_tgt == nullptr || n_micro < 1) return set_err(h, GPT2_EINVAL, "bad train_step arguments");
   if (B < 1 || T < 1 || B > h->maxB || T > h->maxT) return set_err(h, GPT2_EINVAL, "B or T out of range");
   const long M = (long)B * T;
+  RET_IF(clear_accumulators(h));
   CU_CHECK(h, cudaMemsetAsync(h->grads, 0, h->nparams * 4, h->stream));
   CU_CHECK(h, cudaMemsetAsync(h->d_loss + 1, 0, 4, h->stream));
   const float scale = 1.f / (float)n_micro;
@@ -180,6 +182,7 @@ int gpt2_set_params(gpt2_t* h, const float* src) {
 
 int gpt2_get_grads(gpt2_t* h, float* dst) {
   if (h == nullptr || dst == nullptr) return GPT2_EINVAL;
+  RET_IF(fold_accumulators(h));
   RET_IF(check_device_flags(h));
   CU_CHECK(h, cudaMemcpy(dst, h->grads, h->nparams * 4, cudaMemcpyDeviceToHost));
   return GPT2_OK;

@@ -22,6 +22,8 @@ struct TensorInfo {
   int decay;
 };
 
+static const size_t NO_OFF = (size_t)-1;  // no parameter
+
 struct LayerOffsets {
   size_t ln1g, ln1b, attnw, attnb, projw, projb, ln2g, ln2b, fcw, fcb, mpw, mpb;
 };
@@ -53,16 +55,39 @@ struct gpt2 {
   float *lse = nullptr, *lnf_mean = nullptr, *lnf_rstd = nullptr;
   float *ce_lse = nullptr, *losses = nullptr, *d_loss = nullptr;
   float* ce_part = nullptr;  // lm_head softmax statistics per (row, 128 columns) (bf16 mode)
-  float* attn_cs = nullptr;  // per-128-row-block column sums of dqkv from the attention backward (bf16 mode)
   bf16* attn_ds = nullptr;   // the attention backward's dS tiles, one layer at a time (bf16 mode)
   int32_t* argmax = nullptr;
 
   // backward scratch
-  float *dres = nullptr, *dln = nullptr, *attn_D = nullptr, *ln_part = nullptr, *cs_part = nullptr;
+  float *dres = nullptr, *dln = nullptr, *attn_D = nullptr;
   bf16* dres_bf = nullptr;
   uint8_t *dbig = nullptr, *dqkv = nullptr, *datt = nullptr;
-  float* splitk_ws = nullptr;
-  size_t splitk_bytes = 0;
+  // bf16 weight gradients of the layers' linear weights accumulate over K
+  // splits into one buffer per split (no per-call reduction); they are folded
+  // into grads, in split order, before anything reads the gradients
+  struct WgradSlots {
+    size_t woff;  // the weight's offset in the parameter arena
+    float* ptr;   // [splits][n]
+    int splits;
+    long n;
+  };
+  std::vector<WgradSlots> wslots;
+  float* slot_buf = nullptr;
+  size_t slot_floats = 0;
+  // per-block partial column sums (LayerNorm dgamma / dbeta / bias of the
+  // projection feeding the residual point, the fc and qkv biases) likewise
+  // accumulate over the micro-steps in one buffer per use, and are reduced in
+  // row order with the fold.  Index: 2l / 2l+1 LayerNorm 1 / 2 of layer l,
+  // 2L the final LayerNorm, 2L+1+l the fc bias, 3L+1+l the qkv bias of layer l.
+  struct PartialSums {
+    float* buf;     // [rows][ncols]
+    int rows, ncols, C;
+    size_t off[3];  // column j sums into grads[off[j / C] + j % C] (NO_OFF: dropped)
+  };
+  std::vector<PartialSums> psums;
+  float* psum_buf = nullptr;
+  size_t psum_floats = 0;
+  bool accum_dirty = false;  // the accumulators hold sums not yet folded into grads
   uint32_t* emb_keys = nullptr;
   float* emb_part = nullptr;
   int sort_cap = 0;
@@ -223,9 +248,9 @@ static void free_all(gpt2* h) {
                   h->ln2,     h->ln1_mean, h->ln1_rstd, h->ln2_mean, h->ln2_rstd, h->qkv,      h->att,
                   h->fcu,     h->fca,     h->lnf,      h->logits,   h->lse,      h->lnf_mean, h->lnf_rstd,
                   h->ce_lse,  h->losses,  h->d_loss,   h->argmax,   h->dres,     h->dln,      h->attn_D,
-                  h->ln_part, h->cs_part, h->dres_bf,  h->dbig,     h->dqkv,     h->datt,     h->splitk_ws,
+                  h->psum_buf, h->dres_bf,  h->dbig,     h->dqkv,     h->datt,     h->slot_buf,
                   h->emb_keys, h->emb_part, h->normbuf, h->d_step, h->norm_part, h->segs,    h->d_bad,    h->tok_dev,
-                  h->tgt_dev, h->ce_part, h->attn_cs, h->attn_ds, h->kv, h->dec_x, h->dec_mean, h->dec_rstd, h->dec_ln,
+                  h->tgt_dev, h->ce_part, h->attn_ds, h->kv, h->dec_x, h->dec_mean, h->dec_rstd, h->dec_ln,
                   h->dec_qkv, h->dec_att, h->dec_u, h->dec_a, h->dec_logits};
   for (void* p : ptrs)
     if (p) cudaFree(p);

@@ -114,7 +114,6 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
   ALLOC(h, h->ce_lse, (size_t)Mx * 4);
   if (h->prec == GPT2_BF16) {
     ALLOC(h, h->ce_part, (size_t)Mx * tcg::ce_halves(h->Vp) * 3 * 4);
-    ALLOC(h, h->attn_cs, (size_t)tcfa::backward_colsum_rows(h->maxB, h->maxT) * 3 * C * 4);
     ALLOC(h, h->attn_ds, (size_t)tcfa::backward_ds_elems(h->maxB, h->maxT, H) * 2);
   }
   ALLOC(h, h->losses, (size_t)Mx * 4);
@@ -133,23 +132,61 @@ static int create_impl(gpt2* h, const gpt2_config* c, uint64_t seed) {
     ALLOC(h, h->attn_D, (size_t)(nb > Mx * H ? nb : Mx * H) * 4);
   }
   {
+    // partial column sums accumulated over the micro-steps (see PartialSums)
     const int rpb = ln_rows_per_block(Mx);
-    const long nblk = (Mx + rpb - 1) / rpb;
-    ALLOC(h, h->ln_part, (size_t)nblk * 3 * C * 4);
+    const int nblk = (int)((Mx + rpb - 1) / rpb);
     const int crpb = colsum_rows_per_block(Mx);
-    const long cblk = (Mx + crpb - 1) / crpb;
-    ALLOC(h, h->cs_part, (size_t)cblk * 4 * C * 4);
+    const int cblk = (int)((Mx + crpb - 1) / crpb);
+    const int qrows = h->prec == GPT2_BF16 ? (int)tcfa::backward_colsum_rows(h->maxB, h->maxT) : cblk;
+    h->psums.resize(4 * L + 1);
+    for (int l = 0; l < L; ++l) {
+      const LayerOffsets& o = h->lo[l];
+      h->psums[2 * l] = {nullptr, nblk, 3 * C, C, {o.ln1g, o.ln1b, l > 0 ? h->lo[l - 1].mpb : NO_OFF}};
+      h->psums[2 * l + 1] = {nullptr, nblk, 3 * C, C, {o.ln2g, o.ln2b, o.projb}};
+      h->psums[2 * L + 1 + l] = {nullptr, cblk, 4 * C, 4 * C, {o.fcb, NO_OFF, NO_OFF}};
+      h->psums[3 * L + 1 + l] = {nullptr, qrows, 3 * C, 3 * C, {o.attnb, NO_OFF, NO_OFF}};
+    }
+    h->psums[2 * L] = {nullptr, nblk, 3 * C, C, {h->lnfg, h->lnfb, h->lo[L - 1].mpb}};
+    size_t total = 0;
+    for (auto& ps : h->psums) total += (size_t)ps.rows * ps.ncols;
+    h->psum_floats = total;
+    ALLOC(h, h->psum_buf, total * 4);
+    CU_CHECK(h, cudaMemsetAsync(h->psum_buf, 0, total * 4, h->stream));
+    size_t at = 0;
+    for (auto& ps : h->psums) {
+      ps.buf = h->psum_buf + at;
+      at += (size_t)ps.rows * ps.ncols;
+    }
   }
   if (h->prec == GPT2_BF16) {
-    // largest split-K scratch over the weight-gradient shapes of the model
-    size_t ws = 0;
-    const int shapes[5][2] = {{3 * C, C}, {C, C}, {4 * C, C}, {C, 4 * C}, {h->Vp, C}};
-    for (auto& s : shapes) {
-      const size_t b = tcg::splitk_workspace_bytes(s[0], s[1], (int)Mx, 0);
-      if (b > ws) ws = b;
+    // per-split accumulators of the weight gradients that the tcgen05 GEMM
+    // splits over the tokens (the lm_head's has tiles enough and goes straight
+    // into grads)
+    size_t total = 0;
+    for (int l = 0; l < L; ++l) {
+      const LayerOffsets& o = h->lo[l];
+      const size_t w[4][3] = {{o.attnw, (size_t)3 * C, (size_t)C},
+                              {o.projw, (size_t)C, (size_t)C},
+                              {o.fcw, (size_t)4 * C, (size_t)C},
+                              {o.mpw, (size_t)C, (size_t)4 * C}};
+      for (auto& x : w) {
+        const int sp = tcg::accum_slot_splits((int)x[1], (int)x[2], (int)Mx);
+        if (sp < 2) continue;
+        const long n = (long)(x[1] * x[2]);
+        h->wslots.push_back({x[0], nullptr, sp, n});
+        total += (size_t)sp * n;
+      }
     }
-    h->splitk_bytes = ws;
-    if (ws) ALLOC(h, h->splitk_ws, ws);
+    h->slot_floats = total;
+    if (total) {
+      ALLOC(h, h->slot_buf, total * 4);
+      CU_CHECK(h, cudaMemsetAsync(h->slot_buf, 0, total * 4, h->stream));
+      size_t at = 0;
+      for (auto& ws : h->wslots) {
+        ws.ptr = h->slot_buf + at;
+        at += (size_t)ws.splits * ws.n;
+      }
+    }
   }
   ALLOC(h, h->emb_keys, (size_t)Mx * 4);
   ALLOC(h, h->emb_part, (size_t)Mx * C * 4);

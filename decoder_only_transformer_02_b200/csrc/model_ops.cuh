@@ -3,7 +3,6 @@
 #pragma once
 #include "model_core.cuh"
 
-static const size_t NO_OFF = (size_t)-1;
 
 // ----------------------------------------------------------------- LayerNorm
 template <typename TO>
@@ -43,21 +42,22 @@ static bool ln_bwd_attr() {
 }
 
 // LayerNorm backward into the running residual gradient h->dres.  dy is fp32
-// [M, C].  Adds dgamma, dbeta and (when dbias_off != NO_OFF) the column sums of
-// the resulting residual gradient into the grads.
+// [M, C].  Its partial column sums (dgamma, dbeta and the bias gradient of the
+// projection feeding this residual point) add into h->psums[inst].
 static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean, const float* rstd, size_t goff,
-                     size_t boff, size_t dbias_off, long M, int accumulate) {
+                     int inst, long M, int accumulate) {
   KTimer kt(h, KC_LN_B, 0.0, (double)M * h->C * (12 + (accumulate ? 4 : 0) + (h->prec == GPT2_BF16 ? 2 : 0)) + 8.0 * M);
   const int rpb = ln_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
   bf16* dbf = h->prec == GPT2_BF16 ? h->dres_bf : nullptr;
+  float* part = h->psums[inst].buf;
   switch (h->C / 128) {
 #define LNB(NV)                                                                                                     \
   case NV:                                                                                                          \
     if (k::LnBwd<NV>::smem_bytes(rpb) > LN_BWD_SMEM_MAX) return set_err(h, GPT2_EINVAL, "layernorm: rows");     \
     if (!ln_bwd_attr<NV>()) return set_err(h, GPT2_ECUDA, "layernorm backward shared memory");                  \
     k::ln_bwd_kernel<NV><<<nblk, (k::LN_BWD_WARPS + 1) * 32, k::LnBwd<NV>::smem_bytes(rpb), h->stream>>>(       \
-        dy, x, mean, rstd, h->P32(goff), h->dres, dbf, (int)M, rpb, accumulate, h->ln_part);                        \
+        dy, x, mean, rstd, h->P32(goff), h->dres, dbf, (int)M, rpb, accumulate, part);                              \
     break;
     LNB(1) LNB(2) LNB(3) LNB(4) LNB(5) LNB(6) LNB(7) LNB(8)
 #undef LNB
@@ -65,10 +65,7 @@ static int op_ln_bwd(gpt2* h, const float* dy, const float* x, const float* mean
       return set_err(h, GPT2_EINVAL, "n_embd must be a multiple of 128 up to 1024");
   }
   LAUNCH_CHECK(h);
-  k::partials_reduce_kernel<<<dim3((3 * h->C + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(
-      h->ln_part, nblk, 3 * h->C, h->C, h->G32(goff), h->G32(boff),
-      dbias_off == NO_OFF ? nullptr : h->G32(dbias_off));
-  LAUNCH_CHECK(h);
+  h->accum_dirty = true;
   return GPT2_OK;
 }
 
@@ -79,7 +76,7 @@ static int tc_call(gpt2* h, tcg::GemmArgs& g) {
   const int r = tcg::gemm(g, h->stream);
   if (r == -1) return set_err(h, GPT2_EINVAL, "matmul: bad shape / stride / alignment");
   if (r != 0) return set_err(h, GPT2_ECUDA, "matmul: tensor map or launch failure");
-  h->launches += (g.epi == tcg::EPI_ACCUM_F32 && g.workspace) ? 2 : 1;
+  h->launches += 1;
   return GPT2_OK;
 }
 static int simt_call(gpt2* h, const simt::Args& a) {
@@ -213,8 +210,12 @@ static int op_lin_wgrad(gpt2* h, const void* dY, long M, int N, const void* X, i
     g.out = h->G32(woff);
     g.ldc = Kin;
     g.epi = tcg::EPI_ACCUM_F32;
-    g.workspace = h->splitk_ws;
-    g.workspace_bytes = h->splitk_bytes;
+    for (const auto& ws : h->wslots)
+      if (ws.woff == woff) {
+        g.slots = ws.ptr;
+        g.slot_splits = ws.splits;
+        h->accum_dirty = true;
+      }
     return tc_call(h, g);
   }
   simt::Args a{};
@@ -233,32 +234,21 @@ static int op_lin_wgrad(gpt2* h, const void* dY, long M, int N, const void* X, i
   return simt_call(h, a);
 }
 
-// grads[boff .. +N] += column sums of a[M, N] (activation type)
-static int op_colsum(gpt2* h, const void* a, long M, int N, size_t boff) {
+// Partial column sums of a[M, N] (activation type), added into
+// h->psums[inst] (folded into the bias gradient later).
+static int op_colsum(gpt2* h, const void* a, long M, int N, int inst) {
   KTimer kt(h, KC_OTHER, 0.0, (double)M * N * h->es);
   const int rpb = colsum_rows_per_block(M);
   const int nblk = (int)((M + rpb - 1) / rpb);
   const int vec = h->prec == GPT2_BF16 ? 8 : 4;
   dim3 grid((N + 32 * vec - 1) / (32 * vec), nblk);
+  float* part = h->psums[inst].buf;
   if (h->prec == GPT2_BF16)
-    k::colsum_partial_kernel<bf16><<<grid, 256, 0, h->stream>>>((const bf16*)a, (int)M, N, rpb, h->cs_part);
+    k::colsum_partial_kernel<bf16><<<grid, 256, 0, h->stream>>>((const bf16*)a, (int)M, N, rpb, part);
   else
-    k::colsum_partial_kernel<float><<<grid, 256, 0, h->stream>>>((const float*)a, (int)M, N, rpb, h->cs_part);
+    k::colsum_partial_kernel<float><<<grid, 256, 0, h->stream>>>((const float*)a, (int)M, N, rpb, part);
   LAUNCH_CHECK(h);
-  k::partials_reduce_kernel<<<dim3((N + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(h->cs_part, nblk, N, N, h->G32(boff), nullptr,
-                                                                   nullptr);
-  LAUNCH_CHECK(h);
-  return GPT2_OK;
-}
-
-// grads[boff .. +3C] += the attention backward's per-block column sums of dqkv
-static int op_attn_bias_reduce(gpt2* h, size_t boff) {
-  KTimer kt(h, KC_OTHER, 0.0, 0.0);
-  const int nblk = (int)tcfa::backward_colsum_rows(h->B, h->T);
-  const int n = 3 * h->C;
-  k::partials_reduce_kernel<<<dim3((n + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(h->attn_cs, nblk, n, n, h->G32(boff), nullptr,
-                                                                  nullptr);
-  LAUNCH_CHECK(h);
+  h->accum_dirty = true;
   return GPT2_OK;
 }
 
@@ -290,9 +280,10 @@ static int op_attn_bwd(gpt2* h, int l) {
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;
   if (h->prec == GPT2_BF16) {
     if (tcfa::backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
-                       h->B, h->T, h->H, h->stream, h->attn_cs, h->attn_ds) != cudaSuccess)
+                       h->B, h->T, h->H, h->stream, h->psums[3 * h->L + 1 + l].buf, h->attn_ds) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention backward launch");
     h->launches += 3;
+    h->accum_dirty = true;
   } else {
     if (attn::naive_backward((const float*)qkv, (const float*)att, (const float*)h->datt, lse, (float*)h->dqkv,
                              h->attn_D, h->B, h->T, h->H, h->C / h->H, h->stream) != cudaSuccess)

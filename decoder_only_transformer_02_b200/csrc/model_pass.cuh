@@ -131,28 +131,24 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
   // lm_head (tied): dwte += dlogits^T xf ; dxf = dlogits wte
   RET_IF(op_lin_wgrad(h, dlog, M, h->Vp, h->lnf, C, h->wte));
   RET_IF(op_lin_dgrad(h, dlog, M, h->Vp, h->wte, C, DG_F32, h->dln, nullptr));
-  RET_IF(op_ln_bwd(h, h->dln, w.res(2 * L), h->lnf_mean, h->lnf_rstd, h->lnfg, h->lnfb, h->lo[L - 1].mpb, M, 0));
+  RET_IF(op_ln_bwd(h, h->dln, w.res(2 * L), h->lnf_mean, h->lnf_rstd, h->lnfg, 2 * L, M, 0));
   for (int l = L - 1; l >= 0; --l) {
     const LayerOffsets& o = h->lo[l];
     // MLP half: x_out = x_mid + mproj(gelu(fc(ln2(x_mid))))
     RET_IF(op_lin_wgrad(h, dres_act, M, C, w.fca(l), 4 * C, o.mpw));
     RET_IF(op_lin_dgrad(h, dres_act, M, C, o.mpw, 4 * C, DG_DGELU, h->dbig, w.fcu(l)));
-    RET_IF(op_colsum(h, h->dbig, M, 4 * C, o.fcb));
+    RET_IF(op_colsum(h, h->dbig, M, 4 * C, 2 * L + 1 + l));
     RET_IF(op_lin_wgrad(h, h->dbig, M, 4 * C, w.ln2(l), C, o.fcw));
     RET_IF(op_lin_dgrad(h, h->dbig, M, 4 * C, o.fcw, C, DG_F32, h->dln, nullptr));
-    RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l + 1), w.ln2m(l), w.ln2r(l), o.ln2g, o.ln2b, o.projb, M, 1));
+    RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l + 1), w.ln2m(l), w.ln2r(l), o.ln2g, 2 * l + 1, M, 1));
     // attention half: x_mid = x_in + proj(attn(qkv(ln1(x_in))))
     RET_IF(op_lin_wgrad(h, dres_act, M, C, w.att(l), C, o.projw));
     RET_IF(op_lin_dgrad(h, dres_act, M, C, o.projw, C, DG_ACT, h->datt, nullptr));
-    RET_IF(op_attn_bwd(h, l));
-    if (h->prec == GPT2_BF16)
-      RET_IF(op_attn_bias_reduce(h, o.attnb));
-    else
-      RET_IF(op_colsum(h, h->dqkv, M, 3 * C, o.attnb));
+    RET_IF(op_attn_bwd(h, l));  // (bf16: with the qkv bias partial sums)
+    if (h->prec != GPT2_BF16) RET_IF(op_colsum(h, h->dqkv, M, 3 * C, 3 * L + 1 + l));
     RET_IF(op_lin_wgrad(h, h->dqkv, M, 3 * C, w.ln1(l), C, o.attnw));
     RET_IF(op_lin_dgrad(h, h->dqkv, M, 3 * C, o.attnw, C, DG_F32, h->dln, nullptr));
-    RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l), w.ln1m(l), w.ln1r(l), o.ln1g, o.ln1b, l > 0 ? h->lo[l - 1].mpb : NO_OFF,
-                     M, 1));
+    RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l), w.ln1m(l), w.ln1r(l), o.ln1g, 2 * l, M, 1));
   }
   // embeddings: dwte[tok] += dx0 (sorted, fixed order), dwpe[t] += sum_b dx0[b, t]
   KTimer kt(h, KC_EMB, 0.0, 8.0 * M * C + 8.0 * T * C);
@@ -164,21 +160,51 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
                                                                           h->sort_cap);
     LAUNCH_CHECK(h);
   }
-  const int eth = C < 256 ? C : 256;
+  const int eth = C / 4;  // one thread per 4 columns (n_embd <= 1024)
   k::embed_bwd_partial_kernel<<<(unsigned)((M + k::EMB_CH - 1) / k::EMB_CH), eth, 0, h->stream>>>(
       h->emb_keys, h->dres, (int)M, C, h->emb_part);
   LAUNCH_CHECK(h);
-  k::embed_bwd_reduce_kernel<<<grid_for(M, 1, 16), eth, 0, h->stream>>>(h->emb_keys, h->emb_part, (int)M, C,
-                                                                        h->Vp, h->G32(h->wte));
+  k::embed_bwd_reduce_kernel<<<(unsigned)M, eth, 0, h->stream>>>(h->emb_keys, h->emb_part, (int)M, C, h->Vp,
+                                                                 h->G32(h->wte));
   LAUNCH_CHECK(h);
-  k::wpe_bwd_kernel<<<grid_for((long)T * C, 256), 256, 0, h->stream>>>(h->dres, B, T, C, h->G32(h->wpe));
+  k::wpe_bwd_kernel<<<grid_for((long)T * C / 4, 256), 256, 0, h->stream>>>(h->dres, B, T, C, h->G32(h->wpe));
   LAUNCH_CHECK(h);
   h->have_bwd_keys = true;
   h->have_targets = false;  // one backward per forward
   return GPT2_OK;
 }
 
+// Fold the accumulators (the per-split weight gradients and the partial
+// column sums) into grads, in a fixed order, and clear them.
+static int fold_accumulators(gpt2* h) {
+  if (!h->accum_dirty) return GPT2_OK;
+  KTimer kt(h, KC_OPT, 0.0, 12.0 * (double)h->slot_floats + 4.0 * (double)h->psum_floats);
+  for (const auto& ws : h->wslots) {
+    k::slot_fold_kernel<<<grid_for(ws.n / 4, 256, 4), 256, 0, h->stream>>>(h->G32(ws.woff), ws.ptr, ws.n, ws.splits);
+    LAUNCH_CHECK(h);
+  }
+  for (const auto& ps : h->psums) {
+    float* o[3];
+    for (int j = 0; j < 3; ++j) o[j] = ps.off[j] == NO_OFF ? nullptr : h->G32(ps.off[j]);
+    k::partials_reduce_kernel<<<dim3((ps.ncols + 31) / 32, k::PR_SPLIT), 256, 0, h->stream>>>(
+        ps.buf, ps.rows, ps.ncols, ps.C, o[0], o[1], o[2]);
+    LAUNCH_CHECK(h);
+  }
+  CU_CHECK(h, cudaMemsetAsync(h->psum_buf, 0, h->psum_floats * 4, h->stream));
+  h->accum_dirty = false;
+  return GPT2_OK;
+}
+// Discard whatever the accumulators hold (with the gradients being zeroed).
+static int clear_accumulators(gpt2* h) {
+  if (!h->accum_dirty) return GPT2_OK;
+  if (h->slot_buf) CU_CHECK(h, cudaMemsetAsync(h->slot_buf, 0, h->slot_floats * 4, h->stream));
+  CU_CHECK(h, cudaMemsetAsync(h->psum_buf, 0, h->psum_floats * 4, h->stream));
+  h->accum_dirty = false;
+  return GPT2_OK;
+}
+
 static int adamw_impl(gpt2* h, float lr, float wd, float b1, float b2, float eps, float clip) {
+  RET_IF(fold_accumulators(h));
   const long n = (long)h->nparams;
   KTimer kt(h, KC_OPT, 0.0, 34.0 * n);
   long per = (n + h->norm_blocks - 1) / h->norm_blocks;
@@ -288,5 +314,6 @@ static int fused_micro_step(gpt2* h, const int32_t* tok, const int32_t* tgt, int
   h->have_targets = false;
   h->logits_valid = false;
   h->have_bwd_keys = true;
+  h->accum_dirty = true;  // its gradients went into the accumulators
   return GPT2_OK;
 }

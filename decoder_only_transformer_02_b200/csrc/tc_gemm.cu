@@ -233,8 +233,9 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
     } break;
     case EPI_RESID_F32:
     case EPI_ACCUM_F32: {
-      const float* rs = (p.epi == EPI_RESID_F32 ? p.resid : reinterpret_cast<const float*>(p.out)) + base;
-      float* o = reinterpret_cast<float*>(p.out) + base;
+      const long soff = p.epi == EPI_ACCUM_F32 ? (long)split * p.split_stride : 0;
+      const float* rs = (p.epi == EPI_RESID_F32 ? p.resid : reinterpret_cast<const float*>(p.out) + soff) + base;
+      float* o = reinterpret_cast<float*>(p.out) + soff + base;
       if (FULL) {
         uint32_t x[4][8];
 #pragma unroll
@@ -343,8 +344,8 @@ __device__ __forceinline__ void epi_ce_chunk(const Params& p, int row, int col0,
 // words) or GELU pre-activation (bf16, 2 x 32-byte words) the caller already
 // loaded into x: the vectorised epilogue of EPI_RESID_F32, EPI_ACCUM_F32 and
 // EPI_DGELU.
-__device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int col0, const uint32_t (&r)[32],
-                                                 const uint32_t (*x)[8]) {
+__device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int col0, int split,
+                                                 const uint32_t (&r)[32], const uint32_t (*x)[8]) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -374,7 +375,7 @@ __device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int c
       v[4 * i + 3] += bb.w;
     }
   }
-  float* o = reinterpret_cast<float*>(p.out) + base;
+  float* o = reinterpret_cast<float*>(p.out) + (p.epi == EPI_ACCUM_F32 ? (long)split * p.split_stride : 0) + base;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
 #pragma unroll
@@ -432,7 +433,9 @@ __device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, 
       uint32_t x[8][8];
       if (pre) {
         if (f32_in) {
-          const float* src = (p.epi == EPI_RESID_F32 ? p.resid : reinterpret_cast<const float*>(p.out)) +
+          const float* src = (p.epi == EPI_RESID_F32
+                                  ? p.resid
+                                  : reinterpret_cast<const float*>(p.out) + (long)split * p.split_stride) +
                              (long)row * p.ldc + col;
 #pragma unroll
           for (int i = 0; i < 8; ++i) ld32(src + 8 * i, x[i]);
@@ -457,9 +460,9 @@ __device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, 
         const int col0 = col + h * 32;
         if (pre) {
           if (f32_in)
-            epi_store_loaded(p, row, col0, r, &x[4 * h]);
+            epi_store_loaded(p, row, col0, split, r, &x[4 * h]);
           else
-            epi_store_loaded(p, row, col0, r, &x[2 * h]);
+            epi_store_loaded(p, row, col0, split, r, &x[2 * h]);
         } else if (row < p.M && col0 < p.N) {
           if (col0 + 32 <= p.N && p.vec32)
             epi_store<true>(p, row, col0, split, r);
@@ -998,6 +1001,16 @@ int choose_splits(int tiles, int kb_total, int units) {
   return best;
 }
 
+int accum_slot_splits(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 1;
+  const int bn = (N <= 128) ? 128 : 256;
+  const bool pair = use_pair_kernel(M, N, bn);
+  const int tiles = pair ? ceil_div(M, 256) * ceil_div(N, 256) : ceil_div(M, BM) * ceil_div(N, bn);
+  const int kbt = ceil_div(K, BK);
+  const int s = choose_splits(tiles, kbt, pair ? num_sms() / 2 : num_sms());
+  return ceil_div(kbt, ceil_div(kbt, s));
+}
+
 size_t splitk_workspace_bytes(int M, int N, int K, int bn) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   if (bn != 128) bn = (N <= 128) ? 128 : 256;
@@ -1059,22 +1072,32 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
     if (g.workspace) ok = ok && al32(g.workspace) && (g.ldc * 4L) % 32 == 0;
     p.vec32 = ok ? 1 : 0;
   }
-  int splits = 1;
-  if (g.epi == EPI_ACCUM_F32 && g.workspace != nullptr) {
-    splits = choose_splits(p.num_m * p.num_n, p.kb_total, pair ? num_sms() / 2 : num_sms());
+  const int units = pair ? num_sms() / 2 : num_sms();
+  int splits = 1;       // K splits
+  bool reduce = false;  // split-K partials in g.workspace, summed into out by a reduction kernel
+  if (g.epi == EPI_ACCUM_F32 && g.slots != nullptr) {
+    // persistent per-split accumulators: no scratch, no reduction
+    if (g.ldc != g.N || (reinterpret_cast<uintptr_t>(g.slots) & 15)) return -1;
+    splits = choose_splits(p.num_m * p.num_n, p.kb_total, units);
+    if (splits > g.slot_splits) splits = g.slot_splits;
+    if (splits < 1) splits = 1;
+    p.out = g.slots;
+    p.split_stride = (long)g.M * g.ldc;
+    p.vec32 = p.vec32 && (reinterpret_cast<uintptr_t>(g.slots) & 31) == 0;
+  } else if (g.epi == EPI_ACCUM_F32 && g.workspace != nullptr && g.ldc == g.N) {
+    splits = choose_splits(p.num_m * p.num_n, p.kb_total, units);
     if (splits > 1 && g.workspace_bytes < (size_t)splits * g.M * g.ldc * sizeof(float)) splits = 1;
+    reduce = splits > 1;
   }
-  if (splits > 1 && g.ldc != g.N) splits = 1;
-  if (splits > 1) {
+  {
+    // every split gets at least one k-block
     const int kps = ceil_div(p.kb_total, splits);
-    splits = ceil_div(p.kb_total, kps);
+    p.splits = ceil_div(p.kb_total, kps);
     p.kb_per_split = kps;
-    p.splits = splits;
+  }
+  if (reduce) {
     p.epi = EPI_PARTIAL_F32;
     p.partial = g.workspace;
-  } else {
-    p.kb_per_split = p.kb_total;
-    p.splits = 1;
   }
   p.total_tiles = p.num_m * p.num_n * p.splits;
   cudaError_t e;
@@ -1089,12 +1112,12 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
                               : launch<256, false>(ta, tb, p, grid, st);
   }
   if (e != cudaSuccess) return -3;
-  if (splits > 1) {
+  if (reduce) {
     const long n = (long)g.M * g.N;
     const long n4 = n / 4;
     int blocks = (int)((n4 + 255) / 256);
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
-    splitk_reduce_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(g.out), g.workspace, n4, n, splits);
+    splitk_reduce_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<float*>(g.out), g.workspace, n4, n, p.splits);
     if (cudaGetLastError() != cudaSuccess) return -3;
   }
   return 0;

@@ -41,6 +41,12 @@ struct GemmArgs {
   size_t workspace_bytes = 0;
   int bn = 0;                   // 0: automatic (256 unless N <= 128), or 128 / 256
   float* ce_part = nullptr;     // EPI_CE_STATS: [M][ce_halves(N)][3] (max, sum of exp(z - max), argmax bits)
+  // EPI_ACCUM_F32 over K splits into persistent per-split accumulators (no
+  // reduction here): split s adds its share of the sum into
+  // slots[s][M][N] (ldc == N); at most slot_splits splits.  The caller folds
+  // the slots into the final sum later, in split order.  out is unused.
+  float* slots = nullptr;
+  int slot_splits = 0;
 };
 
 // Number of softmax-statistics partials per row that EPI_CE_STATS writes.
@@ -62,12 +68,16 @@ struct Params {
   int vec32;  // 1: every 32-column chunk is 32-byte aligned (vector epilogue)
   float* ce_part;
   int ce_nh;
+  long split_stride;  // EPI_ACCUM_F32: elements between the accumulators of consecutive splits (0: one)
 };
 
 // Returns 0 on success, -1 bad arguments, -2 tensor-map encode failure, -3 launch failure.
 int gemm(const GemmArgs& g, cudaStream_t stream);
 // Bytes of split-K scratch that an EPI_ACCUM_F32 call of this shape would use.
 size_t splitk_workspace_bytes(int M, int N, int K, int bn);
+// K splits that an EPI_ACCUM_F32 call of this shape uses with per-split
+// accumulators (1: none needed).
+int accum_slot_splits(int M, int N, int K);
 int choose_splits(int tiles, int kb_total, int units);
 
 }  // namespace tcg

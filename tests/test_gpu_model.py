@@ -177,6 +177,28 @@ def test_graph_replay_equals_eager_launches():
         np.testing.assert_array_equal(ga, gb)
 
 
+def test_graph_replay_with_split_accumulators_equals_eager():
+    """Two optimizer steps of three micro-steps each, with the weight
+    gradients split over 1024 tokens into per-split accumulators: the second
+    step replays every micro-step from the CUDA graph, and the accumulators
+    must still be folded into the gradients before the update.  The
+    parameters must be the very bits of all-eager launches."""
+    cfgd = dict(n_layer=2, n_head=4, n_embd=256, vocab_size=500, padded_vocab=512, block_size=256)
+    params = {}
+    for graphs in (False, True):
+        G, O, cfg, m = make(cfgd, 4, 256, 1, seed=9)
+        m.set_graphs(graphs)
+        for step in range(2):
+            m.zero_grad()
+            for k, (tok, tgt) in enumerate(batch("zipf", cfg.vocab_size, 4, 256, 90 + 10 * step, n=3)):
+                m.forward_backward(dev(tok), dev(tgt), 1.0 / 3)
+            m.adamw_step(6e-4)
+        params[graphs] = m.get_params()
+        m.close()
+    assert not np.array_equal(params[False], 0)
+    np.testing.assert_array_equal(params[False], params[True])
+
+
 def test_bf16_accumulated_optimizer_step_matches_oracle():
     """The accumulated optimizer step in bf16 mode: four micro-steps with
     distinct batches at loss scale 1/4 (the first eager, the second captured
@@ -188,7 +210,9 @@ def test_bf16_accumulated_optimizer_step_matches_oracle():
     Bars: |dloss| <= 1e-2, per-tensor gradient cosine >= 0.999 (read before
     the step), norm within 1%, per-tensor cosine of the update dp >= 0.999."""
     cfgd = dict(n_layer=2, n_head=4, n_embd=256, vocab_size=500, padded_vocab=512, block_size=256)
-    B, T, n_micro, lr, clip = 2, 128, 4, 6e-4, 1e-2
+    # (1024 tokens per micro-step: the layers' weight gradients are split over
+    # the tokens into per-split accumulators, folded before they are read)
+    B, T, n_micro, lr, clip = 4, 256, 4, 6e-4, 1e-2
     G, O, cfg, m = make(cfgd, B, T, 1, seed=5)
     flat = O.init_params(cfg, 5).astype(np.float32)
     m.set_params(flat)
