@@ -42,7 +42,12 @@ WORKLOADS = {
 }
 N_PARAMS = 124_475_904
 L, C, V, VP = 12, 768, 50257, 50304
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "bf16_sustained_sm_mhz": 1300.0}  # the sustained figure settles at about 1.3 GHz
+# DRAM bytes (read + write) per launch of the 2-SM GEMM kernel, averaged over
+# the captured launches of the ncu launch list of the default workload
+# (dram__bytes_read.sum + dram__bytes_write.sum, one pass, this build)
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 def flops_per_token(T: int) -> float:
@@ -319,10 +324,18 @@ def run_ours(args):
     roofline = {"kernel": "tc_gemm_kernel (tcgen05 bf16 GEMM, all matmul shapes of the step)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
-                "traffic": None,
+                "traffic": GEMM_TRAFFIC_BYTES_PER_LAUNCH,
+                "traffic_unit": "bytes per launch (mean over the class's launches in an ncu launch list)",
                 "timed_by": f"CUDA events around every launch, {prof_steps} instrumented steps of the same "
                             f"sequence run eagerly right after the timed region ({prof_ms:.1f} ms/step instrumented)",
                 "per_launch": {"flops": g["flops"] / g["ops"], "ms": g["ms"] / g["ops"]}}
+
+    # the GEMM rate per SM clock against the sustained peak's own clock
+    peak_mhz = peaks.get("bf16_sustained_sm_mhz") or peaks.get("sm_mhz_sustained")
+    if clk and clk.get("sm_mhz") and peak_mhz:
+        roofline["frac_per_clock"] = (achieved / clk["sm_mhz"]) / (peak / peak_mhz)
+        roofline["frac_per_clock_note"] = (f"TFLOP/s per median SM MHz ({clk['sm_mhz']:.0f}) over the sustained "
+                                           f"peak per its own SM MHz ({peak_mhz:.0f})")
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -166,21 +166,29 @@ __global__ void embed_bwd_reduce_kernel(const uint32_t* __restrict__ keys, const
 
 
 // g[i] += slots[0][i] + slots[1][i] + ... (in split order), and the slots
-// are cleared for the next accumulation.  n % 4 == 0.
+// are cleared for the next accumulation.  n % 4 == 0, splits <= SLOT_MAX; all
+// of a thread's loads are issued before its adds and stores.
+constexpr int SLOT_MAX = 16;
 __global__ void slot_fold_kernel(float* __restrict__ g, float* __restrict__ slots, long n, int splits) {
   const long n4 = n / 4;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float4 v[SLOT_MAX];
+#pragma unroll
+    for (int s = 0; s < SLOT_MAX; ++s)
+      if (s < splits) v[s] = reinterpret_cast<const float4*>(slots + s * n)[i];
     float4 acc = reinterpret_cast<const float4*>(g)[i];
-    for (int s = 0; s < splits; ++s) {
-      float4* q = reinterpret_cast<float4*>(slots + s * n) + i;
-      const float4 v = *q;
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-      *q = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+#pragma unroll
+    for (int s = 0; s < SLOT_MAX; ++s)
+      if (s < splits) {
+        acc.x += v[s].x;
+        acc.y += v[s].y;
+        acc.z += v[s].z;
+        acc.w += v[s].w;
+      }
     reinterpret_cast<float4*>(g)[i] = acc;
+#pragma unroll
+    for (int s = 0; s < SLOT_MAX; ++s)
+      if (s < splits) reinterpret_cast<float4*>(slots + s * n)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
