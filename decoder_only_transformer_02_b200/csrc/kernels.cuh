@@ -271,8 +271,8 @@ __global__ void ln_fwd_kernel(const float* __restrict__ x, const float* __restri
 //   linear layer whose output is this residual point).
 // A CTA owns a fixed range of rows.  One producer thread streams them into
 // shared memory with bulk asynchronous copies (dy, x and the incoming dres of
-// LN_BWD_WARPS rows per stage, LnBwd<NV>::STAGES stages), so the bytes in
-// flight do not depend on registers; each compute warp takes one row of a
+// LN_BWD_WARPS consecutive rows per stage, one copy per array, LnBwd<NV>::STAGES
+// stages), so the bytes in flight do not depend on registers; each compute warp takes one row of a
 // stage, reads it from shared memory, writes dres / dres_bf to global memory,
 // and keeps its columns' sums in registers.  At the end the warps' sums are
 // combined in warp order.  Rows per CTA: a multiple of LN_BWD_WARPS.
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(32 * (LN_BWD_WARPS + 1), 1)
   using L = LnBwd<NV>;
   constexpr int C = L::C, S = L::STAGES, W = LN_BWD_WARPS;
   extern __shared__ float4 ln_smem4[];
-  float* stage = reinterpret_cast<float*>(ln_smem4);  // [S][W][dy | x | dres]
+  float* stage = reinterpret_cast<float*>(ln_smem4);  // [S][dy | x | dres][W][C]
   float* mr = stage + S * L::STAGE_FLOATS;              // mean [rows_per_block], rstd [rows_per_block]
   uint64_t* full = reinterpret_cast<uint64_t*>(mr + 2 * rows_per_block);
   uint64_t* empty = full + S;
@@ -327,15 +327,15 @@ __global__ void __launch_bounds__(32 * (LN_BWD_WARPS + 1), 1)
           ok = false;
           break;
         }
+        // the batch's rows are contiguous in each array: one copy per array
         const int nr = min(W, nrows - k * W);
-        tcg::mbar_expect_tx(&full[s], (uint32_t)(nr * (accumulate ? 3 : 2) * C * 4));
-        for (int w = 0; w < nr; ++w) {
-          const long row = r0 + (long)k * W + w;
-          float* dst = stage + (long)s * L::STAGE_FLOATS + w * L::ROW;
-          tcfa::bulk_load(tcg::smem_u32(dst), dy + row * C, C * 4, &full[s]);
-          tcfa::bulk_load(tcg::smem_u32(dst + C), x + row * C, C * 4, &full[s]);
-          if (accumulate) tcfa::bulk_load(tcg::smem_u32(dst + 2 * C), dres + row * C, C * 4, &full[s]);
-        }
+        const uint32_t bytes = (uint32_t)(nr * C * 4);
+        const long row = r0 + (long)k * W;
+        float* dst = stage + (long)s * L::STAGE_FLOATS;
+        tcg::mbar_expect_tx(&full[s], (accumulate ? 3 : 2) * bytes);
+        tcfa::bulk_load(tcg::smem_u32(dst), dy + row * C, bytes, &full[s]);
+        tcfa::bulk_load(tcg::smem_u32(dst + W * C), x + row * C, bytes, &full[s]);
+        if (accumulate) tcfa::bulk_load(tcg::smem_u32(dst + 2 * W * C), dres + row * C, bytes, &full[s]);
       }
       if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
       tcfa::drain_ring(full, S, (uint32_t)issued);
@@ -355,14 +355,15 @@ __global__ void __launch_bounds__(32 * (LN_BWD_WARPS + 1), 1)
       const int ri = k * W + warp;
       if (ri < nrows) {
         const long row = r0 + ri;
-        const float4* src = reinterpret_cast<const float4*>(stage + (long)s * L::STAGE_FLOATS + warp * L::ROW);
+        // this warp's row of the stage's dy, x and dres blocks
+        const float4* src = reinterpret_cast<const float4*>(stage + (long)s * L::STAGE_FLOATS + warp * C);
         const float mu = mr[ri], rs = mr[rows_per_block + ri];
         float4 dyv[NV], xv[NV];
         float s1 = 0.f, s2 = 0.f;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
           dyv[i] = src[lane + 32 * i];
-          const float4 xr = src[C / 4 + lane + 32 * i];
+          const float4 xr = src[W * C / 4 + lane + 32 * i];
           xv[i] = make_float4((xr.x - mu) * rs, (xr.y - mu) * rs, (xr.z - mu) * rs, (xr.w - mu) * rs);
           const float d0 = dyv[i].x * g[i].x, d1 = dyv[i].y * g[i].y, d2 = dyv[i].z * g[i].z, d3 = dyv[i].w * g[i].w;
           s1 += d0 + d1 + d2 + d3;
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(32 * (LN_BWD_WARPS + 1), 1)
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
           const int c4 = lane + 32 * i;
-          const float4 rv = accumulate ? src[C / 2 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 rv = accumulate ? src[W * C / 2 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
           float4 o;
           o.x = rv.x + rs * (dyv[i].x * g[i].x - s1 - xv[i].x * s2);
           o.y = rv.y + rs * (dyv[i].y * g[i].y - s1 - xv[i].y * s2);
