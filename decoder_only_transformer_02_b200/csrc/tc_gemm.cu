@@ -169,10 +169,21 @@ __device__ __forceinline__ void st32(void* p, uint32_t a, uint32_t b, uint32_t c
                "r"(f), "r"(g), "r"(h)
                : "memory");
 }
+// (read-once streams: the residual, accumulator and pre-activation inputs of
+// the epilogues do not allocate in L1, which keeps the bias there)
 __device__ __forceinline__ void ld32(const void* p, uint32_t (&r)[8]) {
-  asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+  asm volatile("ld.global.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "l"(p));
+}
+// bias loads: every lane of a warp reads the same 16 bytes, tile after tile,
+// so they are kept in L1 with the highest priority
+__device__ __forceinline__ float4 ldg_keep(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.nc.L1::evict_last.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
 }
 __device__ __forceinline__ void st_bf16x16(bf16* o, const float* v) {
   st32(o, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]),
@@ -198,7 +209,7 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
       const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 b = __ldg(b4 + i);
+        const float4 b = ldg_keep(b4 + i);
         v[4 * i] += b.x;
         v[4 * i + 1] += b.y;
         v[4 * i + 2] += b.z;
@@ -368,7 +379,7 @@ __device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int c
     const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 bb = __ldg(b4 + i);
+      const float4 bb = ldg_keep(b4 + i);
       v[4 * i] += bb.x;
       v[4 * i + 1] += bb.y;
       v[4 * i + 2] += bb.z;
