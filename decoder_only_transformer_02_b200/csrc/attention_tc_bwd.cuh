@@ -1016,8 +1016,9 @@ static inline long backward_colsum_rows(int B, int T) { return (long)B * ((T + B
 // T)][3C] fp32 partial column sums of dqkv, added to what it holds (summing
 // them over the rows gives the qkv bias gradient).
 //  ds given (backward_ds_elems(B, T, H) bf16, 16-byte aligned): ld_kernel forms
-//     lse*log2(e) and D, dkdv_kernel forms P and dS once per score and stores
-//     dS, dq_mma_kernel reads it back for dQ (three launches).
+//     lse*log2(e) and D (unless ld_ready: the caller already wrote them into
+//     ld), dkdv_kernel forms P and dS once per score and stores dS,
+//     dq_mma_kernel reads it back for dQ (three launches, or two).
 //  ds null: dq_kernel forms D and dQ from recomputed scores, then dkdv_kernel
 //     (two launches, no scratch beyond ld).
 // Both routes run the same arithmetic on every score (the products of S and
@@ -1025,7 +1026,7 @@ static inline long backward_colsum_rows(int B, int T) { return (long)B * ((T + B
 // the same order), so their results agree bit for bit.
 static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, bf16* dqkv,
                                    float* ld, int B, int T, int H, cudaStream_t st, float* colsum = nullptr,
-                                   bf16* ds = nullptr) {
+                                   bf16* ds = nullptr, bool ld_ready = false) {
   static DeviceOnce once;
   cudaError_t e = run_once_per_device(once, [] {
     cudaError_t r = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKV_SMEM);
@@ -1050,7 +1051,9 @@ static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16*
     CUtensorMap tds;
     if (make_tmap(&tds, ds, BT, backward_ds_elems(B, T, H) / BT, BT, 64, 64) != 0) return cudaErrorInvalidValue;
     const long n = (long)B * ((T + BT - 1) / BT) * BT * H;
-    if (((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(dout)) & 31) == 0)
+    if (ld_ready) {
+      // lse*log2(e) and D are already in ld (formed by the kernel that wrote dout)
+    } else if (((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(dout)) & 31) == 0)
       ld_kernel<true><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
     else
       ld_kernel<false><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);

@@ -153,11 +153,13 @@ static int op_lm_head_ce(gpt2* h, long M) {
   return tc_call(h, g);
 }
 
-enum DgradKind { DG_F32, DG_ACT, DG_DGELU };  // fp32 out / activation-typed out / x gelu'(aux)
+// fp32 out / activation-typed out / x gelu'(aux) / bf16 out plus the attention
+// backward's lse*log2(e) and D rows of layer `aux_layer` (the output is dO)
+enum DgradKind { DG_F32, DG_ACT, DG_DGELU, DG_ACT_ROWDOT };
 
 // dX[M,Kin] = dY[M,N] W[N,Kin]
 static int op_lin_dgrad(gpt2* h, const void* dY, long M, int N, size_t woff, int Kin, DgradKind kind, void* out,
-                        const void* aux) {
+                        const void* aux, int aux_layer = -1) {
   KTimer kt(h, KC_GEMM, 2.0 * M * N * Kin, 0.0);
   if (h->prec == GPT2_BF16) {
     tcg::GemmArgs g;
@@ -174,6 +176,15 @@ static int op_lin_dgrad(gpt2* h, const void* dY, long M, int N, size_t woff, int
     g.ldc = Kin;
     g.epi = kind == DG_F32 ? tcg::EPI_F32 : (kind == DG_ACT ? tcg::EPI_BF16 : tcg::EPI_DGELU);
     g.aux = (const bf16*)aux;
+    if (kind == DG_ACT_ROWDOT) {
+      // aux: the layer's attention output O; the row dots D = rowsum(dO * O)
+      // and lse*log2(e) go to the attention backward's scratch
+      g.epi = tcg::EPI_ROWDOT;
+      g.aux = (const bf16*)(h->att + (size_t)aux_layer * h->Mmax() * h->C * h->es);
+      g.rd_out = h->attn_D;
+      g.rd_lse = h->lse + (size_t)aux_layer * h->Mmax() * h->H;
+      g.rd_T = h->T;
+    }
     return tc_call(h, g);
   }
   simt::Args a{};
@@ -273,6 +284,10 @@ static int op_attn_fwd(gpt2* h, int l) {
   return GPT2_OK;
 }
 
+// T a multiple of 128: the attention-output projection's dgrad forms the
+// backward's lse*log2(e) and D rows (EPI_ROWDOT) instead of a separate kernel
+static bool attn_rows_fused(const gpt2* h) { return h->prec == GPT2_BF16 && h->T % 128 == 0; }
+
 static int op_attn_bwd(gpt2* h, int l) {
   KTimer kt(h, KC_ATTN_B, 4.0 * h->B * (double)h->T * h->T * h->C, 0.0);
   uint8_t* qkv = h->qkv + (size_t)l * h->Mmax() * 3 * h->C * h->es;
@@ -280,9 +295,10 @@ static int op_attn_bwd(gpt2* h, int l) {
   float* lse = h->lse + (size_t)l * h->Mmax() * h->H;
   if (h->prec == GPT2_BF16) {
     if (tcfa::backward((const bf16*)qkv, (const bf16*)att, (const bf16*)h->datt, lse, (bf16*)h->dqkv, h->attn_D,
-                       h->B, h->T, h->H, h->stream, h->psums[3 * h->L + 1 + l].buf, h->attn_ds) != cudaSuccess)
+                       h->B, h->T, h->H, h->stream, h->psums[3 * h->L + 1 + l].buf, h->attn_ds,
+                       attn_rows_fused(h)) != cudaSuccess)
       return set_err(h, GPT2_ECUDA, "attention backward launch");
-    h->launches += 3;
+    h->launches += attn_rows_fused(h) ? 2 : 3;
     h->accum_dirty = true;
   } else {
     if (attn::naive_backward((const float*)qkv, (const float*)att, (const float*)h->datt, lse, (float*)h->dqkv,

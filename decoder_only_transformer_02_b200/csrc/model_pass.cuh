@@ -143,7 +143,8 @@ static int backward_impl(gpt2* h, float loss_scale, bool fused) {
     RET_IF(op_ln_bwd(h, h->dln, w.res(2 * l + 1), w.ln2m(l), w.ln2r(l), o.ln2g, 2 * l + 1, M, 1));
     // attention half: x_mid = x_in + proj(attn(qkv(ln1(x_in))))
     RET_IF(op_lin_wgrad(h, dres_act, M, C, w.att(l), C, o.projw));
-    RET_IF(op_lin_dgrad(h, dres_act, M, C, o.projw, C, DG_ACT, h->datt, nullptr));
+    RET_IF(op_lin_dgrad(h, dres_act, M, C, o.projw, C, attn_rows_fused(h) ? DG_ACT_ROWDOT : DG_ACT, h->datt, nullptr,
+                        l));
     RET_IF(op_attn_bwd(h, l));  // (bf16: with the qkv bias partial sums)
     if (h->prec != GPT2_BF16) RET_IF(op_colsum(h, h->dqkv, M, 3 * C, 3 * L + 1 + l));
     RET_IF(op_lin_wgrad(h, h->dqkv, M, 3 * C, w.ln1(l), C, o.attnw));

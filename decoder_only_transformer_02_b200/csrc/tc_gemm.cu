@@ -356,11 +356,26 @@ __device__ __forceinline__ void epi_ce_chunk(const Params& p, int row, int col0,
 // loaded into x: the vectorised epilogue of EPI_RESID_F32, EPI_ACCUM_F32 and
 // EPI_DGELU.
 __device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int col0, int split,
-                                                 const uint32_t (&r)[32], const uint32_t (*x)[8]) {
+                                                 const uint32_t (&r)[32], const uint32_t (*x)[8],
+                                                 float (&dot)[4]) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
   const long base = (long)row * p.ldc + col0;
+  if (p.epi == EPI_ROWDOT) {
+    // the stored bf16 values, and their products with aux in four chains
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+      const float2 a = unpack_bf16x2(w[i]), o = unpack_bf16x2(x[i / 8][i % 8]);
+      dot[i & 3] = fmaf(a.x, o.x, fmaf(a.y, o.y, dot[i & 3]));
+    }
+    bf16* ob = reinterpret_cast<bf16*>(p.out) + base;
+    st32(ob, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st32(ob + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+    return;
+  }
   if (p.epi == EPI_DGELU) {
     bf16* o = reinterpret_cast<bf16*>(p.out) + base;
 #pragma unroll
@@ -434,7 +449,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, 
     }
   } else {
     const bool f32_in = p.epi == EPI_RESID_F32 || p.epi == EPI_ACCUM_F32;
-    const bool loads = (f32_in || p.epi == EPI_DGELU) && p.vec32 && row < p.M;
+    const bool loads = (f32_in || p.epi == EPI_DGELU || p.epi == EPI_ROWDOT) && p.vec32 && row < p.M;
     // 64 accumulator columns per TMEM wait; the buffer is handed back to the
     // MMA warp as soon as its last columns are in registers
 #pragma unroll 1
@@ -457,6 +472,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, 
         }
       }
       if (j == 0 && !wait_acc()) return false;
+      float dot[4] = {0.f, 0.f, 0.f, 0.f};  // EPI_ROWDOT: the chunk's 64 columns are one group
       // the chunk's two 32-column halves, one TMEM load and wait each
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -471,15 +487,22 @@ __device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, 
         const int col0 = col + h * 32;
         if (pre) {
           if (f32_in)
-            epi_store_loaded(p, row, col0, split, r, &x[4 * h]);
+            epi_store_loaded(p, row, col0, split, r, &x[4 * h], dot);
           else
-            epi_store_loaded(p, row, col0, split, r, &x[2 * h]);
+            epi_store_loaded(p, row, col0, split, r, &x[2 * h], dot);
         } else if (row < p.M && col0 < p.N) {
           if (col0 + 32 <= p.N && p.vec32)
             epi_store<true>(p, row, col0, split, r);
           else
             epi_store<false>(p, row, col0, split, r);
         }
+      }
+      if (p.epi == EPI_ROWDOT && pre) {
+        const int T = p.rd_T, H = p.N / 64, nqb = T / 128;
+        const int b = row / T, q = row % T, hd = col / 64;
+        float* ld = p.rd_out + (((long)b * H + hd) * nqb + q / 128) * 256 + q % 128;
+        ld[0] = p.rd_lse[((long)b * H + hd) * T + q] * 1.4426950408889634f;
+        ld[128] = (dot[0] + dot[1]) + (dot[2] + dot[3]);
       }
     }
   }
@@ -1070,18 +1093,28 @@ int gemm(const GemmArgs& g, cudaStream_t st) {
   p.ldc = g.ldc;
   p.ce_part = g.ce_part;
   p.ce_nh = ce_halves(g.N);
+  p.rd_out = g.rd_out;
+  p.rd_lse = g.rd_lse;
+  p.rd_T = g.rd_T;
+  if (g.epi == EPI_ROWDOT && (g.rd_out == nullptr || g.rd_lse == nullptr || g.aux == nullptr || g.rd_T <= 0 ||
+                              g.rd_T % 128 != 0 || g.N % 64 != 0 || g.M % g.rd_T != 0 || g.ldc != g.N || g.bias))
+    return -1;
   if (g.epi == EPI_CE_STATS && (g.ce_part == nullptr || bn != 256)) return -1;
   {
     // 32-byte vector epilogue: every 32-column chunk of every row (and of the
     // residual / aux / split-K partial buffers) must start on 32 bytes
-    const size_t es = (g.epi == EPI_BF16 || g.epi == EPI_GELU || g.epi == EPI_DGELU || g.epi == EPI_CE_STATS) ? 2 : 4;
+    const size_t es =
+        (g.epi == EPI_BF16 || g.epi == EPI_GELU || g.epi == EPI_DGELU || g.epi == EPI_CE_STATS || g.epi == EPI_ROWDOT)
+            ? 2
+            : 4;
     auto al32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31) == 0; };
     bool ok = (g.ldc * (long)es) % 32 == 0 && al32(g.out);
     if (g.epi == EPI_RESID_F32) ok = ok && al32(g.resid);
     if (g.epi == EPI_GELU) ok = ok && al32(g.out2);
-    if (g.epi == EPI_DGELU) ok = ok && al32(g.aux);
+    if (g.epi == EPI_DGELU || g.epi == EPI_ROWDOT) ok = ok && al32(g.aux);
     if (g.workspace) ok = ok && al32(g.workspace) && (g.ldc * 4L) % 32 == 0;
     p.vec32 = ok ? 1 : 0;
+    if (g.epi == EPI_ROWDOT && !ok) return -1;  // its row dots are formed on the vector path only
   }
   const int units = pair ? num_sms() / 2 : num_sms();
   int splits = 1;       // K splits

@@ -16,6 +16,8 @@ enum Epi : int {
   EPI_PARTIAL_F32 = 6,  // internal: split-K partial tiles
   EPI_CE_STATS = 7,     // internal: out(bf16) = acc, plus per-(row, half tile) softmax statistics of the
                         // stored (bf16-rounded) values into ce_part
+  EPI_ROWDOT = 8,       // out(bf16) = acc, plus per (row, 64 columns) the dot product of the stored
+                        // values with aux (bf16, same layout), into rd_out (see GemmArgs)
 };
 
 // Logical problem: D[M,N] = sum_k A[m,k] B[n,k].
@@ -47,6 +49,14 @@ struct GemmArgs {
   // the slots into the final sum later, in split order.  out is unused.
   float* slots = nullptr;
   int slot_splits = 0;
+  // EPI_ROWDOT (N = 64 H, M = B T, T % 128 == 0): for row m = b T + q and
+  // column group h, rd_out[((b H + h) nqb + q / 128) 256 + 128 + q % 128] =
+  // sum of out[m][64h + c] * aux[m][64h + c] over c, and the entry 128 below
+  // it = rd_lse[(b H + h) T + q] * log2(e) (nqb = T / 128): the rows of
+  // lse*log2(e) and D = rowsum(dO * O) of the attention backward.
+  float* rd_out = nullptr;
+  const float* rd_lse = nullptr;
+  int rd_T = 0;
 };
 
 // Number of softmax-statistics partials per row that EPI_CE_STATS writes.
@@ -69,6 +79,9 @@ struct Params {
   float* ce_part;
   int ce_nh;
   long split_stride;  // EPI_ACCUM_F32: elements between the accumulators of consecutive splits (0: one)
+  float* rd_out;      // EPI_ROWDOT
+  const float* rd_lse;
+  int rd_T;
 };
 
 // Returns 0 on success, -1 bad arguments, -2 tensor-map encode failure, -3 launch failure.
