@@ -417,14 +417,15 @@ def sub_record_workload(G, S, torch, name, peaks, steps=3, warmup=3):
 
 def sub_record_attention(G, torch, peaks, reps=5):
     """The standalone causal attention workload: B=8, H=12, d=64, T in
-    {1024, 2048, 4096}, forward and backward timed separately with CUDA events
-    around each call; L2 flushed (256 MB write) before every timed call."""
+    {1024, 2048, 4096} and, beyond it, 8192; forward and backward timed
+    separately with CUDA events around each call; L2 flushed (256 MB write)
+    before every timed call."""
     from decoder_only_transformer_02_b200.synthetic import normal_array
     st = torch.cuda.current_stream()
     flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
     out = {"B": 8, "H": 12, "d": 64, "flops_convention": "causal: fwd 2*B*H*T^2*d, bwd 2x fwd",
            "l2": "flushed before every timed call"}
-    for T in (1024, 2048, 4096):
+    for T in (1024, 2048, 4096, 8192):
         B, H = 8, 12
         Cc = 64 * H
         qkv = torch.from_numpy(normal_array((B, T, 3 * Cc), 3)).to(torch.bfloat16).cuda()
