@@ -3,36 +3,38 @@
 // With P = exp(S/sqrt(d) - lse) and D_q = sum_d dO_q . O_q:
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dK = dS^T Q / sqrt(d),
 //   dQ = dS K / sqrt(d).
-// Two deterministic kernels (no atomics), each persistent with one CTA per SM
-// and 128 x 128 score tiles.  A CTA takes work items in a fixed order, longest
-// first, and its pipeline runs across item boundaries (the next item's tiles
-// load and its first MMAs run while the current item's results are written).
-//  dq_kernel (runs first): an item is 128 queries of one (batch, head); it
-//     walks the 128-key blocks up to its last query:
-//       S = Q K_j^T, dP = dO V_j^T        (M=128 queries, N=128 keys, K=64)
-//       dS = P * (dP - D)                  (sixteen compute warps, bf16 into TMEM)
-//       dQ += dS K_j                       (A = dS read from TMEM, K=128 keys)
-//     It also forms D for its queries (from the dO tile in shared memory and
-//     the rows of O; one warp per lane quarter, shared with the other three
-//     through shared memory) and writes lse*log2(e) and D per 128-query block
-//     into a padded fp32 array (+inf / 0 past T) that dkdv_kernel streams by
-//     bulk copy.
+// Deterministic (no atomics).  The tile kernels are persistent with one CTA
+// per SM and 128 x 128 score tiles; a CTA takes work items longest first in
+// a snake order, and its pipeline runs across item boundaries (the next
+// item's tiles load and its first MMAs run while the current item's results
+// are written).
+//  ld_kernel: lse*log2(e) and D per query, padded to whole 128-query blocks
+//     (+inf / 0 past T), unless the caller already formed them.
 //  dkdv_kernel: an item is 128 keys of one (batch, head); it walks the
 //     128-query blocks that reach them:
 //       S^T = K Q_i^T, dP^T = V dO_i^T     (M=128 keys, N=128 queries, K=64)
-//       P^T, dS^T                          (bf16 into TMEM)
+//       P^T, dS^T                          (sixteen compute warps, bf16 into TMEM)
 //       dV += P^T dO_i, dK += dS^T Q_i     (A from TMEM, K=128 queries)
-// The score tiles never touch shared memory: S and dP are read from TMEM into
-// registers, and P / dS go back into TMEM as the A operand of the next MMAs.
-// Warp 0 streams the operand tiles through a 4-stage TMA ring, warp 1 issues
-// the MMAs (one thread), warps 2..17 do the element-wise math: warps w, w+4,
-// w+8 and w+12 share TMEM lane quarter w%4 (one row each) and take the four
-// 32-column quarters of the tile, so every SM sub-partition has four warps to
-// hide the TMEM and shared-memory latencies with.  While the warps work on tile j, the tensor cores already run
-// S_{j+1} and dP_{j+1} (and the accumulating MMAs of tile j-1).  Both kernels
-// can also write per-(128-row block, lane quarter) column sums of what they
-// store (the qkv bias gradient).  Every wait is bounded; the waits that drain
-// a CTA's own copies and MMAs before it exits have their own fixed limit.
+//     and stores every dS^T block as a bf16 tile: the compute warps write it
+//     into a swizzled staging tile in shared memory, a store warp issues the
+//     TMA stores.
+//  dq_mma_kernel: dQ_i = sum_j dS_ij K_j / sqrt(d) from the stored tiles, so
+//     no score is formed twice.
+// Without room for the dS tiles (the no-allocation entry point), dq_kernel
+// forms D and dQ from recomputed scores per 128-query block instead:
+//       S = Q K_j^T, dP = dO V_j^T, dS = P * (dP - D), dQ += dS K_j
+// and dkdv_kernel runs without its stores.  The score tiles go from TMEM to
+// registers and back into TMEM as the A operand of the next MMAs.  Warp 0
+// streams the operand tiles through a TMA ring, warp 1 issues the MMAs (one
+// thread), warps 2..17 do the element-wise math: warps w, w+4, w+8 and w+12
+// share TMEM lane quarter w%4 (one row each) and take the four 32-column
+// quarters of the tile, so every SM sub-partition has four warps to hide the
+// TMEM and shared-memory latencies with.  While the warps work on tile j, the
+// tensor cores already run the next tile's score MMAs (and the accumulating
+// MMAs of tile j-1).  The kernels can also add per-(128-row block, lane
+// quarter) column sums of what they store (the qkv bias gradient) into a
+// caller's buffer.  Every wait is bounded; the waits that drain a CTA's own
+// copies and MMAs before it exits have their own fixed limit.
 #pragma once
 #include "attention.cuh"
 #include "attention_tc.cuh"
@@ -434,6 +436,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
 // staging tile of dS^T for its TMA store (four 64x64 boxes, [key half][query
 // half], 128-byte swizzled rows).
 constexpr int DKV_STAGES = 3;
+constexpr int DKV_STORE_WARP = 2 + BW_CWARPS;           // the warp that issues the dS^T TMA stores
+constexpr int DKV_THREADS = BW_THREADS + 32;
 constexpr int DKV_KV_OFF = 0;                              // buffer b: K at +2b*TILE, V at +(2b+1)*TILE
 constexpr int DKV_STAGE_BYTES = 2 * TILE + LD_FLOATS * 4;
 constexpr int DKV_RING_OFF = 4 * TILE;                     // stage s: Q, dO, lse2/D
@@ -445,7 +449,7 @@ constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
 constexpr uint32_t DKV_T_S = 0, DKV_T_DP = 128, DKV_T_DV = 256, DKV_T_DK = 320, DKV_T_P = 384, DKV_T_DS = 448;
 static_assert(DKV_STAGE_BYTES % 1024 == 0, "ring stages keep the 1024-byte swizzle alignment");
 
-__global__ void __launch_bounds__(BW_THREADS, 1)
+__global__ void __launch_bounds__(DKV_THREADS, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_ds, const float* __restrict__ ld_in, bf16* __restrict__ dqkv,
                 float* __restrict__ colsum, int store_ds, int T, int H, int BH, float scale, float sl2) {
@@ -610,6 +614,36 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       tc_commit(drain);
       if (!mbar_wait_drain(drain, 0)) set_device_err(DERR_WAIT_TIMEOUT);
     }
+  } else if (warp == DKV_STORE_WARP) {
+    if (lane == 0 && store_ds) {
+      // ------------------------------------------------- dS^T store warp
+      // once the compute warps have written a block's dS^T into the staging
+      // tile: four TMA stores to tile (bh, query block i, key block kb), and
+      // the staging tile is handed back once the stores have read it
+      uint32_t g = 0;
+      bool ok = true;
+      for (int k = 0, w = snake_item(0); ok && w < nitems; w = snake_item(++k)) {
+        int kb, bh;
+        item(w, kb, bh);
+        const int nblk = nqb - kb;
+        for (int n = 0; n < nblk; ++n, ++g) {
+          const int i = kb + n;
+          if (!mbar_wait(st_full, g & 1u)) {
+            ok = false;
+            break;
+          }
+          const int y = (bh * (nqb * (nqb + 1) / 2) + i * (i + 1) / 2 + kb) * BT;
+#pragma unroll
+          for (int bx = 0; bx < 4; ++bx)
+            tma_store_2d(&tm_ds, (bx & 1) * 64, y + (bx >> 1) * 64, smem_u32(smem + DKV_DS_OFF + bx * 8192));
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(st_free);
+        }
+      }
+      if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
+      bulk_wait0();  // the dS^T stores are complete before the CTA exits
+    }
   } else {
     // ---------------------------------------------------- compute warps
     const int qw = warp & 3;
@@ -670,15 +704,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
           }
         }
         if (store_ds) {
-          // dS^T of this block for dq_mma_kernel, tile (bh, query block i,
-          // key block kb): written into the swizzled staging tile, then one
-          // thread stores it with TMA.  The staging tile is reused once the
-          // previous tile's store has read it.
-          const bool elected = warp == 2 && lane == 0;
-          if (elected && g >= 1) {
-            bulk_wait_read0();
-            mbar_arrive(st_free);
-          }
+          // dS^T of this block for dq_mma_kernel: written into the swizzled
+          // staging tile once the store warp's previous TMA store has read it
           if (!warp_wait(st_free, (g & 1u) ^ 1u)) {
             ok = false;
             break;
@@ -692,18 +719,6 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(st_full);
-          if (elected) {
-            if (!mbar_wait(st_full, g & 1u)) {
-              set_device_err(DERR_WAIT_TIMEOUT);
-            } else {
-              const int y = (bh * (nqb * (nqb + 1) / 2) + i * (i + 1) / 2 + kb) * BT;
-#pragma unroll
-              for (int bx = 0; bx < 4; ++bx)
-                tma_store_2d(&tm_ds, (bx & 1) * 64, y + (bx >> 1) * 64, smem_u32(smem + DKV_DS_OFF + bx * 8192));
-              bulk_commit();
-            }
-          }
-          __syncwarp();
         }
         // the previous step's dV / dK MMAs have read P^T and dS^T
         if (g >= 1 && !warp_wait(p_free, (g - 1) & 1u)) {
@@ -753,7 +768,6 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
       }
     }
     if (!ok) set_device_err(DERR_WAIT_TIMEOUT);
-    if (warp == 2 && lane == 0) bulk_wait0();  // the dS^T stores are complete before the CTA exits
   }
   __syncthreads();
   if (warp == 1) {
@@ -1057,11 +1071,11 @@ static inline cudaError_t backward(const bf16* qkv, const bf16* out, const bf16*
       ld_kernel<true><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
     else
       ld_kernel<false><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(out, dout, lse, ld, B, T, H);
-    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, tds, ld, dqkv, colsum, 1, T, H, B * H, scale, sl2);
+    dkdv_kernel<<<grid, DKV_THREADS, DKV_SMEM, st>>>(tq, td, tds, ld, dqkv, colsum, 1, T, H, B * H, scale, sl2);
     dq_mma_kernel<<<grid, 192, DQM_SMEM, st>>>(tds, tq, dqkv, colsum, T, H, B * H, scale);
   } else {
     dq_kernel<<<grid, BW_THREADS, DQ_SMEM, st>>>(tq, td, out, lse, ld, dqkv, colsum, T, H, B * H, scale, sl2);
-    dkdv_kernel<<<grid, BW_THREADS, DKV_SMEM, st>>>(tq, td, tq, ld, dqkv, colsum, 0, T, H, B * H, scale, sl2);
+    dkdv_kernel<<<grid, DKV_THREADS, DKV_SMEM, st>>>(tq, td, tq, ld, dqkv, colsum, 0, T, H, B * H, scale, sl2);
   }
   return cudaGetLastError();
 }
