@@ -747,8 +747,12 @@ __device__ __forceinline__ void tc_commit_pair_local(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
+// (CTA-scope release: what the MMA issuer needs ordered before it reuses the
+// accumulator are the warp's TMEM loads, which tcgen05.wait::ld and
+// tcgen05.fence::before_thread_sync already order; a cluster-scope release
+// would also wait for the warp's global stores to be acknowledged)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 template <bool CE>
