@@ -130,6 +130,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bit.
@@ -311,6 +319,62 @@ __device__ __forceinline__ void epi_store(const Params& p, int row, int col0, in
   }
 }
 
+// The epilogues that read no memory besides the bias (EPI_BF16, EPI_F32,
+// EPI_PARTIAL_F32, EPI_GELU) on 16 consecutive columns [col0, col0+16) of one
+// row.  Vector path (32-byte accesses) when all 16 lie inside N; the caller
+// has checked p.vec32.
+__device__ __forceinline__ void epi_store16(const Params& p, int row, int col0, int split, const uint32_t (&r)[16]) {
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  const long base = (long)row * p.ldc + col0;
+  const bool bias = p.bias != nullptr && p.epi != EPI_PARTIAL_F32;
+  if (col0 + 16 > p.N) {
+    for (int i = 0; i < 16 && col0 + i < p.N; ++i) {
+      const float x = v[i] + (bias ? __ldg(p.bias + col0 + i) : 0.f);
+      if (p.epi == EPI_BF16) {
+        reinterpret_cast<bf16*>(p.out)[base + i] = f2bf(x);
+      } else if (p.epi == EPI_GELU) {
+        const float u = bf2f(f2bf(x));  // the stored pre-activation, as rounded
+        reinterpret_cast<bf16*>(p.out)[base + i] = f2bf(u);
+        p.out2[base + i] = f2bf(gelu_tanh<true>(u));
+      } else {
+        (p.epi == EPI_F32 ? reinterpret_cast<float*>(p.out) : p.partial + (long)split * p.M * p.ldc)[base + i] = x;
+      }
+    }
+    return;
+  }
+  if (bias) {
+    const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 b = ldg_keep(b4 + i);
+      v[4 * i] += b.x;
+      v[4 * i + 1] += b.y;
+      v[4 * i + 2] += b.z;
+      v[4 * i + 3] += b.w;
+    }
+  }
+  if (p.epi == EPI_BF16) {
+    st_bf16x16(reinterpret_cast<bf16*>(p.out) + base, v);
+  } else if (p.epi == EPI_GELU) {
+    // u rounded to bf16 once; gelu of the rounded u
+    uint32_t wu[8], wg[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      wu[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+      const float2 u = unpack_bf16x2(wu[e]);
+      wg[e] = pack_bf16x2(gelu_tanh<true>(u.x), gelu_tanh<true>(u.y));
+    }
+    st32(reinterpret_cast<bf16*>(p.out) + base, wu[0], wu[1], wu[2], wu[3], wu[4], wu[5], wu[6], wu[7]);
+    st32(p.out2 + base, wg[0], wg[1], wg[2], wg[3], wg[4], wg[5], wg[6], wg[7]);
+  } else {
+    float* o = (p.epi == EPI_F32 ? reinterpret_cast<float*>(p.out) : p.partial + (long)split * p.M * p.ldc) + base;
+    st_f32x8(o, v);
+    st_f32x8(o + 8, v + 8);
+  }
+}
+
 // Softmax statistics epilogue: the 64 accumulator columns [col0, col0+64) of
 // one row are rounded to bf16 and stored (the logits), and their statistics
 // (maximum, sum of exp(z - max), lowest index of the maximum), computed from
@@ -449,7 +513,34 @@ __device__ __forceinline__ bool epilogue_tile(const Params& p, int row, int nb, 
     }
   } else {
     const bool f32_in = p.epi == EPI_RESID_F32 || p.epi == EPI_ACCUM_F32;
-    const bool loads = (f32_in || p.epi == EPI_DGELU || p.epi == EPI_ROWDOT) && p.vec32 && row < p.M;
+    const bool in_loads = f32_in || p.epi == EPI_DGELU || p.epi == EPI_ROWDOT;
+    if (!in_loads && p.vec32) {
+      // 16 accumulator columns per TMEM load, each load issued while the
+      // previous 16 columns are processed
+      constexpr int NP = CHUNKS * 4;
+      const int colw = nb * BN + cbase;
+      uint32_t pa[16], pb[16];
+      if (!wait_acc()) return false;
+      tmem_ld16(tbase + cbase, pa);
+      tmem_wait_ld();
+#pragma unroll 1
+      for (int q = 0; q < NP; q += 2) {
+        tmem_ld16(tbase + cbase + 16 * (q + 1), pb);
+        if (row < p.M && colw + 16 * q < p.N) epi_store16(p, row, colw + 16 * q, split, pa);
+        tmem_wait_ld();
+        if (q + 2 < NP) {
+          tmem_ld16(tbase + cbase + 16 * (q + 2), pa);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release();
+        }
+        if (row < p.M && colw + 16 * (q + 1) < p.N) epi_store16(p, row, colw + 16 * (q + 1), split, pb);
+        if (q + 2 < NP) tmem_wait_ld();
+      }
+      return true;
+    }
+    const bool loads = in_loads && p.vec32 && row < p.M;
     // 64 accumulator columns per TMEM wait; the buffer is handed back to the
     // MMA warp as soon as its last columns are in registers
 #pragma unroll 1
