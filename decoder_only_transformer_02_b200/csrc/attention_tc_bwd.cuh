@@ -444,9 +444,17 @@ constexpr int DKV_RING_OFF = 4 * TILE;                     // stage s: Q, dO, ls
 constexpr int DKV_DS_OFF = DKV_RING_OFF + DKV_STAGES * DKV_STAGE_BYTES;
 constexpr int DKV_BAR_OFF = DKV_DS_OFF + 2 * TILE;
 constexpr int DKV_SMEM = DKV_BAR_OFF + 256 + 1024;
-// TMEM columns: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
-// P^T (bf16 pairs) [384,448), dS^T (bf16 pairs) [448,512)
-constexpr uint32_t DKV_T_S = 0, DKV_T_DP = 128, DKV_T_DV = 256, DKV_T_DK = 320, DKV_T_P = 384, DKV_T_DS = 448;
+// TMEM columns: three 128-column score regions, then dV [384,448) and dK
+// [448,512).  Block g of a CTA's sequence puts S^T in region g%3 and dP^T in
+// region (g+1)%3; once both are in registers, P^T and dS^T (bf16 pairs) go
+// back into S^T's region, each warp into the 32 columns it read: P^T of its
+// 32 queries in the first 16, dS^T in the last 16 (so the 16-query K step kk
+// of the dV / dK MMAs reads columns 32(kk/2) + 8(kk%2) and 16 further on).
+// The MMAs run in issue order, so a region is rewritten only after the MMAs
+// that read it, and the compute warps need not wait for the previous block's
+// dV / dK MMAs before writing P^T and dS^T.
+constexpr uint32_t DKV_T_DV = 384, DKV_T_DK = 448;
+__device__ __forceinline__ uint32_t dkv_region(uint32_t g) { return 128u * (g % 3u); }
 static_assert(DKV_STAGE_BYTES % 1024 == 0, "ring stages keep the 1024-byte swizzle alignment");
 
 __global__ void __launch_bounds__(DKV_THREADS, 1)
@@ -462,9 +470,12 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
   uint64_t* qd_empty = qd_full + DKV_STAGES;  // DKV_STAGES
   uint64_t* s_full = qd_empty + DKV_STAGES;   // S^T and dP^T in TMEM
   uint64_t* s_free = s_full + 1;             // count BW_CWARPS
-  uint64_t* p_full = s_free + 1;             // count BW_CWARPS: P^T and dS^T in TMEM
-  uint64_t* p_free = p_full + 1;             // the dV / dK MMAs have read them
-  uint64_t* acc_done = p_free + 1;           // the item's dV / dK are complete
+  // p_full: P^T and dS^T in TMEM, count BW_CWARPS, one per block parity (the
+  // compute warps no longer wait for the issuer between blocks, so with a
+  // single barrier they could complete a second phase before it waits on the
+  // first)
+  uint64_t* p_full = s_free + 1;             // 2
+  uint64_t* acc_done = p_full + 2;           // the item's dV / dK are complete
   uint64_t* drain = acc_done + 1;
   uint64_t* st_full = drain + 1;             // count BW_CWARPS: the dS^T staging tile is written
   uint64_t* st_free = st_full + 1;           // the previous tile's TMA store has read the staging tile
@@ -486,8 +497,8 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, BW_CWARPS);
-    mbar_init(p_full, BW_CWARPS);
-    mbar_init(p_free, 1);
+    mbar_init(&p_full[0], BW_CWARPS);
+    mbar_init(&p_full[1], BW_CWARPS);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     mbar_init(st_full, BW_CWARPS);
@@ -558,7 +569,7 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
       int pn = 0, plast = 0;  // step g-1: block index within its item, last block of it?
       bool ok = true;
       auto acc_step = [&](uint32_t gp, int np, int last) -> bool {
-        if (!mbar_wait(p_full, gp & 1u)) return false;
+        if (!mbar_wait(&p_full[gp & 1u], (gp >> 1) & 1u)) return false;
         tc_fence_after();
         const int s = gp % DKV_STAGES;
         const uint32_t qa = smem_u32(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES);
@@ -566,11 +577,11 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
           const uint32_t acc = (np > 0 || kk > 0) ? 1u : 0u;
-          tc_mma_ts(tmem + DKV_T_DV, tmem + DKV_T_P + kk * 8, make_sdesc(doa + kk * 2048, 1), id_acc, acc);
-          tc_mma_ts(tmem + DKV_T_DK, tmem + DKV_T_DS + kk * 8, make_sdesc(qa + kk * 2048, 1), id_acc, acc);
+          const uint32_t pa = tmem + dkv_region(gp) + (kk >> 1) * 32 + (kk & 1) * 8;
+          tc_mma_ts(tmem + DKV_T_DV, pa, make_sdesc(doa + kk * 2048, 1), id_acc, acc);
+          tc_mma_ts(tmem + DKV_T_DK, pa + 16, make_sdesc(qa + kk * 2048, 1), id_acc, acc);
         }
         tc_commit(&qd_empty[s]);
-        tc_commit(p_free);
         if (last) tc_commit(acc_done);
         return true;
       };
@@ -595,8 +606,9 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
           const uint32_t doa = qa + TILE;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
-            tc_mma(tmem + DKV_T_S, make_sdesc(ka + kk * 32, 0), make_sdesc(qa + kk * 32, 0), id_s, kk > 0 ? 1u : 0u);
-            tc_mma(tmem + DKV_T_DP, make_sdesc(va + kk * 32, 0), make_sdesc(doa + kk * 32, 0), id_s,
+            tc_mma(tmem + dkv_region(g), make_sdesc(ka + kk * 32, 0), make_sdesc(qa + kk * 32, 0), id_s,
+                   kk > 0 ? 1u : 0u);
+            tc_mma(tmem + dkv_region(g + 1), make_sdesc(va + kk * 32, 0), make_sdesc(doa + kk * 32, 0), id_s,
                    kk > 0 ? 1u : 0u);
           }
           tc_commit(s_full);
@@ -666,26 +678,19 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
         }
         tc_fence_after();
         uint32_t sv[32], dv[32];
-        tmem_ld32(tl + DKV_T_S + cq * 32, sv);
-        tmem_ld32(tl + DKV_T_DP + cq * 32, dv);
+        tmem_ld32(tl + dkv_region(g) + cq * 32, sv);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        tmem_ld32(tl + dkv_region(g + 1) + cq * 32, dv);  // (lands while P is formed)
         const int q0 = i * BT + cq * 32;          // first query of this warp's columns
         const bool diag = q0 < kb * BT + BT - 1;  // some query of the columns precedes some key
         const float* ldl =
             reinterpret_cast<const float*>(smem + DKV_RING_OFF + s * DKV_STAGE_BYTES + 2 * TILE) + cq * 32;
-        // P^T and dS^T of this block, packed to bf16 pairs in place
+        // P^T in fp32, in place of S^T
 #pragma unroll
         for (int c = 0; c < 32; c += 8) {
           const float4 la = *reinterpret_cast<const float4*>(ldl + c);
           const float4 lb = *reinterpret_cast<const float4*>(ldl + c + 4);
-          const float4 da = *reinterpret_cast<const float4*>(ldl + BT + c);
-          const float4 db = *reinterpret_cast<const float4*>(ldl + BT + c + 4);
           const float l8[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-          const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-          float p[8], ds[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float a = fmaf(__uint_as_float(sv[c + e]), sl2, -l8[e]);
@@ -694,8 +699,24 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
                            ? ex2_fma(a)
                            : ex2f(a);
             if (diag && (q0 + c + e < key)) pe = 0.f;
-            p[e] = pe;
-            ds[e] = pe * (__uint_as_float(dv[c + e]) - d8[e]);
+            sv[c + e] = __float_as_uint(pe);
+          }
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // dS^T, then P^T and dS^T packed to bf16 pairs in place
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          const float4 da = *reinterpret_cast<const float4*>(ldl + BT + c);
+          const float4 db = *reinterpret_cast<const float4*>(ldl + BT + c + 4);
+          const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          float p[8], ds[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = __uint_as_float(sv[c + e]);
+            ds[e] = p[e] * (__uint_as_float(dv[c + e]) - d8[e]);
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -720,18 +741,13 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(st_full);
         }
-        // the previous step's dV / dK MMAs have read P^T and dS^T
-        if (g >= 1 && !warp_wait(p_free, (g - 1) & 1u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st16(tl + DKV_T_P + cq * 16, sv);
-        tmem_st16(tl + DKV_T_DS + cq * 16, dv);
+        // into the 32 columns of S^T's region that this warp has read
+        tmem_st16(tl + dkv_region(g) + cq * 32, sv);
+        tmem_st16(tl + dkv_region(g) + cq * 32 + 16, dv);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[g & 1u]);
       }
       if (!ok) break;
       // item epilogue: dV, dK (scaled) and their column sums.  The next item's
