@@ -25,6 +25,23 @@ struct Views {
 
 // fuse: the softmax gradient (scaled by loss_scale / M) overwrites the logits
 // in the same pass that computes the loss
+// The embedding backward's (token, position) sort needs only the ids: it runs
+// on the side stream, forked just before the cross-entropy pass, whose many
+// small CTAs share the SMs with its one CTA (the persistent GEMM and attention
+// kernels of the forward would wait for the SM it holds); the backward joins
+// it before the embedding scatter-add.
+static int fork_embedding_sort(gpt2* h, bool with_targets) {
+  if (!with_targets || h->timing) return GPT2_OK;
+  CU_CHECK(h, cudaEventRecord(h->ev_fork, h->stream));
+  CU_CHECK(h, cudaStreamWaitEvent(h->side_stream, h->ev_fork, 0));
+  k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->side_stream>>>(h->tok_dev, (int)h->M(), h->Vp,
+                                                                             h->emb_keys, h->sort_cap);
+  LAUNCH_CHECK(h);
+  CU_CHECK(h, cudaEventRecord(h->ev_sorted, h->side_stream));
+  h->sort_pending = true;
+  return GPT2_OK;
+}
+
 static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, int T, bool fuse, float loss_scale) {
   if (tok == nullptr) return set_err(h, GPT2_EINVAL, "tokens pointer is NULL");
   if (B < 1 || T < 1 || B > h->maxB || T > h->maxT)
@@ -36,24 +53,17 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
   const long M = h->M();
   const int C = h->C, L = h->L;
   Views w{h};
+  if (h->sort_pending) {
+    // a sort forked by an earlier forward that no backward joined still reads
+    // the ids: join it before they are overwritten
+    CU_CHECK(h, cudaStreamWaitEvent(h->stream, h->ev_sorted, 0));
+    h->sort_pending = false;
+  }
   // keep private copies of the ids: the backward pass reads them again
   if (tok != h->tok_dev) CU_CHECK(h, cudaMemcpyAsync(h->tok_dev, tok, M * 4, cudaMemcpyDeviceToDevice, h->stream));
   if (tgt && tgt != h->tgt_dev)
     CU_CHECK(h, cudaMemcpyAsync(h->tgt_dev, tgt, M * 4, cudaMemcpyDeviceToDevice, h->stream));
   const int32_t* dtgt = tgt ? h->tgt_dev : nullptr;
-  if (dtgt != nullptr && !h->timing) {
-    // the embedding backward's (token, position) sort needs only the ids: run
-    // it on the side stream while the forward runs; the backward joins it
-    CU_CHECK(h, cudaEventRecord(h->ev_fork, h->stream));
-    CU_CHECK(h, cudaStreamWaitEvent(h->side_stream, h->ev_fork, 0));
-    k::sort_keys_kernel<<<1, 1024, (size_t)h->sort_cap * 4, h->side_stream>>>(h->tok_dev, (int)M, h->Vp,
-                                                                               h->emb_keys, h->sort_cap);
-    LAUNCH_CHECK(h);
-    CU_CHECK(h, cudaEventRecord(h->ev_sorted, h->side_stream));
-    h->sort_pending = true;
-  } else {
-    h->sort_pending = false;
-  }
 
   {
     KTimer kt(h, KC_EMB, 0.0, 12.0 * M * C);
@@ -80,6 +90,7 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
     // cross-entropy pass only merges them and streams the row once for the
     // gradient
     RET_IF(op_lm_head_ce(h, M));
+    RET_IF(fork_embedding_sort(h, dtgt != nullptr));
     KTimer kt(h, KC_CE, 0.0, (double)M * h->Vp * 2 * (fuse ? 2 : 0) + (double)M * tcg::ce_halves(h->Vp) * 12);
     k::ce_finish_kernel<<<(unsigned)M, k::CEF_THREADS, 0, h->stream>>>(
         (bf16*)h->logits, h->ce_part, tcg::ce_halves(h->Vp), dtgt, h->Vp, h->ce_lse, dtgt ? h->losses : nullptr,
@@ -87,6 +98,7 @@ static int forward_impl(gpt2* h, const int32_t* tok, const int32_t* tgt, int B, 
     LAUNCH_CHECK(h);
   } else {
     RET_IF(op_lin_fwd(h, h->lnf, M, C, h->wte, h->Vp, NO_OFF, LIN_NOBIAS, h->logits, nullptr, nullptr));
+    RET_IF(fork_embedding_sort(h, dtgt != nullptr));
     const size_t smem = (size_t)h->Vp * h->es;
     KTimer kt(h, KC_CE, 0.0, (double)M * h->Vp * h->es * (fuse ? 2 : 1));
     k::ce_kernel<float><<<(unsigned)M, 1024, smem, h->stream>>>((float*)h->logits, dtgt, h->Vp, h->ce_lse,
