@@ -56,16 +56,32 @@ __device__ __forceinline__ float tanh_fast(float x) {
 // GELU, tanh form: 0.5*u*(1+tanh(sqrt(2/pi)*(u+0.044715*u^3)))
 #define GELU_K 0.7978845608028654f
 #define GELU_A 0.044715f
+// FAST (the bf16 GEMM epilogues): tanh.approx, and the polynomials
+// factored into fused multiply-adds,
+//   t = u (K + K A u^2),  gelu = h + h tanh(t) with h = u / 2,
+//   gelu' = (1 + th) / 2 + (1 - th^2) u (K/2 + 3 K A u^2 / 2);
+// otherwise (the fp32 parity mode) tanhf and the formulas as written.
 template <bool FAST>
 __device__ __forceinline__ float gelu_tanh(float u) {
+  if (FAST) {
+    const float th = tanh_fast(u * fmaf(GELU_K * GELU_A, u * u, GELU_K));
+    const float h = 0.5f * u;
+    return fmaf(h, th, h);
+  }
   float t = GELU_K * (u + GELU_A * u * u * u);
-  float th = FAST ? tanh_fast(t) : tanhf(t);
+  float th = tanhf(t);
   return 0.5f * u * (1.0f + th);
 }
 template <bool FAST>
 __device__ __forceinline__ float gelu_tanh_grad(float u) {
+  if (FAST) {
+    const float u2 = u * u;
+    const float th = tanh_fast(u * fmaf(GELU_K * GELU_A, u2, GELU_K));
+    const float q = u * fmaf(1.5f * GELU_K * GELU_A, u2, 0.5f * GELU_K);
+    return fmaf(q, fmaf(-th, th, 1.0f), fmaf(0.5f, th, 0.5f));
+  }
   float t = GELU_K * (u + GELU_A * u * u * u);
-  float th = FAST ? tanh_fast(t) : tanhf(t);
+  float th = tanhf(t);
   return 0.5f * (1.0f + th) + 0.5f * u * (1.0f - th * th) * GELU_K * (1.0f + 3.0f * GELU_A * u * u);
 }
 
