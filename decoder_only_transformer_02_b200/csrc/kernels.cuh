@@ -218,48 +218,61 @@ __global__ void wpe_bwd_kernel(const float* __restrict__ dx, int B, int T, int C
 // mean/variance, biased variance, eps 1e-5.  Writes y (bf16 or fp32) and the
 // row's mean and rstd.
 template <int NV, typename TO>
-__global__ void ln_fwd_kernel(const float* __restrict__ x, const float* __restrict__ gam, const float* __restrict__ bet,
-                              TO* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int M) {
+__global__ void __launch_bounds__(256, 2) ln_fwd_kernel(const float* __restrict__ x, const float* __restrict__ gam,
+                                                     const float* __restrict__ bet, TO* __restrict__ y,
+                                                     float* __restrict__ mean, float* __restrict__ rstd, int M) {
   constexpr int C = 128 * NV;
   const int lane = threadIdx.x & 31;
-  const long row = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5;
+  const long nw = (long)gridDim.x * (blockDim.x >> 5);  // warps in the grid: the row stride
+  long row = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5;
   if (row >= M) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + row * C);
   float4 v[NV];
-  float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    v[i] = xr[lane + 32 * i];
-    s += v[i].x + v[i].y + v[i].z + v[i].w;
-  }
-  const float mu = warp_sum(s) * (1.f / C);
-  float q = 0.f;
+  for (int i = 0; i < NV; ++i) v[i] = reinterpret_cast<const float4*>(x + row * C)[lane + 32 * i];
+  for (;;) {
+    // the warp's next row loads while this one is normalised
+    const long next = row + nw;
+    float4 vn[NV];
+    if (next < M) {
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const float a = v[i].x - mu, b = v[i].y - mu, c = v[i].z - mu, d = v[i].w - mu;
-    q += a * a + b * b + c * c + d * d;
-  }
-  const float var = warp_sum(q) * (1.f / C);
-  const float rs = rsqrtf(var + 1e-5f);
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = 4 * (lane + 32 * i);
-    const float4 gg = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
-    const float4 bb = reinterpret_cast<const float4*>(bet)[lane + 32 * i];
-    const float o0 = (v[i].x - mu) * rs * gg.x + bb.x;
-    const float o1 = (v[i].y - mu) * rs * gg.y + bb.y;
-    const float o2 = (v[i].z - mu) * rs * gg.z + bb.z;
-    const float o3 = (v[i].w - mu) * rs * gg.w + bb.w;
-    if constexpr (sizeof(TO) == 2) {
-      uint2 w = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
-      *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * C + c) = w;
-    } else {
-      *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * C + c) = make_float4(o0, o1, o2, o3);
+      for (int i = 0; i < NV; ++i) vn[i] = reinterpret_cast<const float4*>(x + next * C)[lane + 32 * i];
     }
-  }
-  if (lane == 0) {
-    mean[row] = mu;
-    rstd[row] = rs;
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) s += v[i].x + v[i].y + v[i].z + v[i].w;
+    const float mu = warp_sum(s) * (1.f / C);
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float a = v[i].x - mu, b = v[i].y - mu, c = v[i].z - mu, d = v[i].w - mu;
+      q += a * a + b * b + c * c + d * d;
+    }
+    const float var = warp_sum(q) * (1.f / C);
+    const float rs = rsqrtf(var + 1e-5f);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * (lane + 32 * i);
+      const float4 gg = reinterpret_cast<const float4*>(gam)[lane + 32 * i];
+      const float4 bb = reinterpret_cast<const float4*>(bet)[lane + 32 * i];
+      const float o0 = (v[i].x - mu) * rs * gg.x + bb.x;
+      const float o1 = (v[i].y - mu) * rs * gg.y + bb.y;
+      const float o2 = (v[i].z - mu) * rs * gg.z + bb.z;
+      const float o3 = (v[i].w - mu) * rs * gg.w + bb.w;
+      if constexpr (sizeof(TO) == 2) {
+        uint2 w = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+        *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(y) + row * C + c) = w;
+      } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + row * C + c) = make_float4(o0, o1, o2, o3);
+      }
+    }
+    if (lane == 0) {
+      mean[row] = mu;
+      rstd[row] = rs;
+    }
+    if (next >= M) break;
+    row = next;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[i] = vn[i];
   }
 }
 

@@ -8,7 +8,10 @@
 template <typename TO>
 static int ln_fwd_dispatch(gpt2* h, const float* x, const float* g, const float* b, TO* y, float* mean, float* rstd,
                            long M) {
-  const int blocks = (int)((M * 32 + 255) / 256);
+  // a warp per row, looping over rows with a stride of the grid's warps: at
+  // most two 8-warp CTAs per SM (what the kernel's registers allow)
+  int blocks = (int)((M * 32 + 255) / 256);
+  if (blocks > 2 * tcg::num_sms()) blocks = 2 * tcg::num_sms();
   switch (h->C / 128) {
 #define LNF(NV) \
   case NV:      \
