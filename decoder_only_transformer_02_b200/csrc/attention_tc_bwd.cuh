@@ -714,9 +714,14 @@ __global__ void __launch_bounds__(DKV_THREADS, 1)
           const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
           float p[8], ds[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 8; e += 2) {
             p[e] = __uint_as_float(sv[c + e]);
-            ds[e] = p[e] * (__uint_as_float(dv[c + e]) - d8[e]);
+            p[e + 1] = __uint_as_float(sv[c + e + 1]);
+            const float2 d = mul2(make_float2(p[e], p[e + 1]),
+                                  sub2(make_float2(__uint_as_float(dv[c + e]), __uint_as_float(dv[c + e + 1])),
+                                       make_float2(d8[e], d8[e + 1])));
+            ds[e] = d.x;
+            ds[e + 1] = d.y;
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {

@@ -40,6 +40,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// Two-wide fp32 arithmetic (sm_100): one instruction for two lanes, each
+// rounded as the scalar operation would be, so results are bit-identical.
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+  return (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
+}
+__device__ __forceinline__ float2 f2_val(uint64_t d) {
+  return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_val(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_val(d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_val(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_val(d);
+}
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(v);
@@ -83,6 +111,24 @@ __device__ __forceinline__ float gelu_tanh_grad(float u) {
   float t = GELU_K * (u + GELU_A * u * u * u);
   float th = tanhf(t);
   return 0.5f * (1.0f + th) + 0.5f * u * (1.0f - th * th) * GELU_K * (1.0f + 3.0f * GELU_A * u * u);
+}
+
+// The FAST forms above on two values with the two-wide instructions: the
+// same operations in the same order on each lane, so the same bits.
+__device__ __forceinline__ float2 gelu_tanh2(float2 u) {
+  const float2 t = mul2(u, fma2(mul2(u, u), make_float2(GELU_K * GELU_A, GELU_K * GELU_A), make_float2(GELU_K, GELU_K)));
+  const float2 th = make_float2(tanh_fast(t.x), tanh_fast(t.y));
+  const float2 h = mul2(make_float2(0.5f, 0.5f), u);
+  return fma2(h, th, h);
+}
+__device__ __forceinline__ float2 gelu_tanh_grad2(float2 u) {
+  const float2 u2 = mul2(u, u);
+  const float2 t = mul2(u, fma2(u2, make_float2(GELU_K * GELU_A, GELU_K * GELU_A), make_float2(GELU_K, GELU_K)));
+  const float2 th = make_float2(tanh_fast(t.x), tanh_fast(t.y));
+  const float2 q = mul2(u, fma2(u2, make_float2(1.5f * GELU_K * GELU_A, 1.5f * GELU_K * GELU_A),
+                                make_float2(0.5f * GELU_K, 0.5f * GELU_K)));
+  const float2 omt = fma2(mul2(th, make_float2(-1.f, -1.f)), th, make_float2(1.f, 1.f));
+  return fma2(q, omt, fma2(make_float2(0.5f, 0.5f), th, make_float2(0.5f, 0.5f)));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

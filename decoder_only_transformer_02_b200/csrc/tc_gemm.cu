@@ -349,10 +349,12 @@ __device__ __forceinline__ void epi_store16(const Params& p, int row, int col0, 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float4 b = ldg_keep(b4 + i);
-      v[4 * i] += b.x;
-      v[4 * i + 1] += b.y;
-      v[4 * i + 2] += b.z;
-      v[4 * i + 3] += b.w;
+      const float2 lo = add2(make_float2(v[4 * i], v[4 * i + 1]), make_float2(b.x, b.y));
+      const float2 hi = add2(make_float2(v[4 * i + 2], v[4 * i + 3]), make_float2(b.z, b.w));
+      v[4 * i] = lo.x;
+      v[4 * i + 1] = lo.y;
+      v[4 * i + 2] = hi.x;
+      v[4 * i + 3] = hi.y;
     }
   }
   if (p.epi == EPI_BF16) {
@@ -363,8 +365,8 @@ __device__ __forceinline__ void epi_store16(const Params& p, int row, int col0, 
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       wu[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-      const float2 u = unpack_bf16x2(wu[e]);
-      wg[e] = pack_bf16x2(gelu_tanh<true>(u.x), gelu_tanh<true>(u.y));
+      const float2 g = gelu_tanh2(unpack_bf16x2(wu[e]));
+      wg[e] = pack_bf16x2(g.x, g.y);
     }
     st32(reinterpret_cast<bf16*>(p.out) + base, wu[0], wu[1], wu[2], wu[3], wu[4], wu[5], wu[6], wu[7]);
     st32(p.out2 + base, wg[0], wg[1], wg[2], wg[3], wg[4], wg[5], wg[6], wg[7]);
@@ -446,9 +448,10 @@ __device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int c
     for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float2 f = unpack_bf16x2(x[hh][e]);
-        v[16 * hh + 2 * e] *= gelu_tanh_grad<true>(f.x);
-        v[16 * hh + 2 * e + 1] *= gelu_tanh_grad<true>(f.y);
+        const float2 d = mul2(make_float2(v[16 * hh + 2 * e], v[16 * hh + 2 * e + 1]),
+                              gelu_tanh_grad2(unpack_bf16x2(x[hh][e])));
+        v[16 * hh + 2 * e] = d.x;
+        v[16 * hh + 2 * e + 1] = d.y;
       }
     st_bf16x16(o, v);
     st_bf16x16(o + 16, v + 16);
@@ -459,17 +462,25 @@ __device__ __forceinline__ void epi_store_loaded(const Params& p, int row, int c
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float4 bb = ldg_keep(b4 + i);
-      v[4 * i] += bb.x;
-      v[4 * i + 1] += bb.y;
-      v[4 * i + 2] += bb.z;
-      v[4 * i + 3] += bb.w;
+      const float2 lo = add2(make_float2(v[4 * i], v[4 * i + 1]), make_float2(bb.x, bb.y));
+      const float2 hi = add2(make_float2(v[4 * i + 2], v[4 * i + 3]), make_float2(bb.z, bb.w));
+      v[4 * i] = lo.x;
+      v[4 * i + 1] = lo.y;
+      v[4 * i + 2] = hi.x;
+      v[4 * i + 3] = hi.y;
     }
   }
   float* o = reinterpret_cast<float*>(p.out) + (p.epi == EPI_ACCUM_F32 ? (long)split * p.split_stride : 0) + base;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[8 * i + e] += __uint_as_float(x[i][e]);
+    for (int e = 0; e < 8; e += 2) {
+      const float2 s =
+          add2(make_float2(v[8 * i + e], v[8 * i + e + 1]),
+               make_float2(__uint_as_float(x[i][e]), __uint_as_float(x[i][e + 1])));
+      v[8 * i + e] = s.x;
+      v[8 * i + e + 1] = s.y;
+    }
     st_f32x8(o + 8 * i, v + 8 * i);
   }
 }
