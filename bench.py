@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch of the 2-SM GEMM kernel, averaged over
 # the captured launches of the ncu launch list of the default workload
 # (dram__bytes_read.sum + dram__bytes_write.sum, one pass, this build)
-GEMM_TRAFFIC_BYTES_PER_LAUNCH = 236.7e6
+GEMM_TRAFFIC_BYTES_PER_LAUNCH = 238.3e6
 
 
 def flops_per_token(T: int) -> float:
