@@ -129,7 +129,7 @@ struct gpt2 {
   bool use_graphs = true;
   cudaStream_t cap_stream = nullptr;
   cudaEvent_t ev_in = nullptr, ev_out = nullptr;
-  // the embedding backward's key sort runs beside the forward on side_stream
+  // the embedding backward's key sort runs beside the cross-entropy pass on side_stream
   cudaStream_t side_stream = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_sorted = nullptr;
   bool sort_pending = false;
