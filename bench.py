@@ -195,6 +195,24 @@ def workload_config(name):
 
 # -------------------------------------------------------------------- ours
 
+def max_over_ranks(x, world, device):
+    """The largest of every rank's x (every rank must call it, in the same
+    order): the slowest rank's time is the job's time."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, steps, tokens_per_step, ms):
+    """Whole-job throughput: the tokens of all ranks (each trains its own
+    replica on its own data) over the slowest rank's time."""
+    return world * steps * tokens_per_step / (ms / 1e3)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -270,11 +288,8 @@ def run_ours(args):
     m.set_timing(False)
     prof_ms = p0.elapsed_time(p1) / prof_steps
     loss = m.last_loss()
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * args.steps * tok_per_step / (ms / 1e3)
+    ms = max_over_ranks(ms, world, "cuda")
+    value = job_tokens_per_s(world, args.steps, tok_per_step, ms)
 
     # end to end through the public C ABI from pinned HOST buffers: every step
     # copies its tokens to the device and reads the loss and norm back
@@ -295,12 +310,8 @@ def run_ours(args):
         e_loss, e_norm = m.train_step(h_tok[s], h_tgt[s], accum, B, T, G.lr_at(2000 + s))
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e = {"value": world * e2e_steps * tok_per_step / (e_ms / 1e3), "unit": "tokens/s",
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+    e2e = {"value": job_tokens_per_s(world, e2e_steps, tok_per_step, e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": int(2 * tok_per_step * 4), "d2h_bytes_per_step": 8,
            "api": "gpt2_train_step (host int32 token/target buffers, pinned)"}
 
