@@ -91,6 +91,13 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        return self.summarize(out)
+
+    @staticmethod
+    def summarize(out: str):
+        """The median SM clock over the busy samples (above half the maximum),
+        the maximum, and every slowdown reason seen active, from the CSV rows
+        of the query above."""
         rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
         if not rows:
             return None

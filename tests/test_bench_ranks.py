@@ -1,8 +1,10 @@
-"""bench.py's multi-rank plumbing, on the CPU: two gloo ranks on 127.0.0.1.
+"""bench.py's host logic, on the CPU.
 
-With N > 1 every rank trains its own replica; the job's time is the slowest
-rank's (an all-reduce MAX that every rank joins), the value counts the tokens
-of all ranks, and the reference arm runs on rank 0 only.
+Multi-rank plumbing as two gloo ranks on 127.0.0.1: with N > 1 every rank
+trains its own replica; the job's time is the slowest rank's (an all-reduce
+MAX that every rank joins), the value counts the tokens of all ranks, and the
+reference arm runs on rank 0 only.  And the clock record the bench line
+carries, from nvidia-smi's rows.
 """
 import argparse
 import datetime
@@ -74,3 +76,25 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     args = argparse.Namespace(workload="t1024", warmup=1, steps=1, gpus=2)
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_clock_summary_takes_busy_samples_and_active_reasons():
+    """The clock record of the bench line, from nvidia-smi's CSV rows
+    (index, sm, max sm, power, active mask, hw, hw thermal, sw thermal, sw power cap)."""
+    import bench
+
+    rows = [
+        "0, 1980, 1965, 150.0, 0x0, Not Active, Not Active, Not Active, Not Active",  # idle sample at start
+        "0, 1590, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1560, 1965, 1000.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1605, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 300, 1965, 80.0, 0x0, Not Active, Not Active, Not Active, Not Active",  # below half the maximum
+    ]
+    rec = bench.ClockSampler.summarize("\n".join(rows))
+    assert rec["sm_max_mhz"] == 1965.0
+    assert rec["sm_mhz"] == 1597.5  # median of 1980, 1590, 1560, 1605
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert rec["samples"] == 5
+    hot = rows[1].replace("Not Active, Not Active, Not Active, Active", "Active, Not Active, Active, Active")
+    assert bench.ClockSampler.summarize(hot)["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+    assert bench.ClockSampler.summarize("") is None
